@@ -1,0 +1,460 @@
+// fg8_host.cu -- the C ABI declared in include/fg8.h: argument checks, tile
+// configuration, TMA descriptor encoding (cached), kernel launches, the scale
+// layout transform and the device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "../../include/fg8.h"
+#include "launch.cuh"
+
+namespace fg8 {
+
+FG8_FOR_EACH_BN(FG8_DECLARE_LAUNCH)
+
+// First error recorded by any GEMM kernel on this device: [0] = code,
+// [1] = (block << 8) | role.  Cleared by fg_get_last_device_status.
+__device__ int g_status[2];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+std::atomic<int> g_num_sms{0};   // 0 = not set: use the device's SM count
+std::atomic<unsigned long long> g_wait_limit_ns{1000000000ull};
+
+struct DeviceInfo {
+    bool ready = false;
+    int sm_count = 0;
+    int cc_major = 0;
+    int regs_ok = -1;   // -1 unknown, 0 kernel build unusable, 1 ok
+    int* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+fg_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return FG_OK;
+    if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver || e == cudaErrorInitializationError)
+        return FG_ERR_NO_DEVICE;
+    return FG_ERR_CUDA;
+}
+
+// Current device, checked to be an sm_100 part; fills *info.
+fg_status current_device(DeviceInfo** info) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_status(e) == FG_OK ? FG_ERR_CUDA : cuda_status(e);
+    }
+    if (dev < 0 || dev >= kMaxDevices) return FG_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_dev_mutex);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return FG_ERR_NO_DEVICE;
+        }
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_status) != cudaSuccess) {
+            cudaGetLastError();
+            return FG_ERR_CUDA;
+        }
+        d.status = static_cast<int*>(addr);
+        d.ready = true;
+    }
+    if (d.cc_major != 10) return FG_ERR_NO_DEVICE;
+    *info = &d;
+    return FG_OK;
+}
+
+int effective_sms(const DeviceInfo& d) {
+    int n = g_num_sms.load();
+    if (n <= 0) {
+        const char* env = std::getenv("FG_NUM_SMS");
+        if (env) n = std::atoi(env);
+    }
+    if (n <= 0 || n > d.sm_count) n = d.sm_count;
+    return n;
+}
+
+// ---- TMA descriptors ---------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return static_cast<EncodeTiledFn>(nullptr);
+        }
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// 3-D E4M3 operand [groups][rows][K] (K innermost), box 128 (K) x box_rows x 1,
+// 128-byte swizzle, zero fill out of bounds.
+struct MapKey {
+    const void* ptr;
+    uint64_t K, rows, groups;
+    uint32_t box_rows;
+    bool operator<(const MapKey& o) const {
+        return std::tie(ptr, K, rows, groups, box_rows) < std::tie(o.ptr, o.K, o.rows, o.groups, o.box_rows);
+    }
+};
+std::map<MapKey, CUtensorMap> g_maps;
+std::mutex g_maps_mutex;
+
+fg_status operand_map(const void* ptr, uint64_t K, uint64_t rows, uint64_t groups, uint32_t box_rows,
+                      CUtensorMap* out) {
+    MapKey key{ptr, K, rows, groups, box_rows};
+    {
+        std::lock_guard<std::mutex> lk(g_maps_mutex);
+        auto it = g_maps.find(key);
+        if (it != g_maps.end()) {
+            *out = it->second;
+            return FG_OK;
+        }
+    }
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return FG_ERR_NO_DEVICE;
+    CUtensorMap m;
+    std::memset(&m, 0, sizeof(m));
+    const cuuint64_t dims[3] = {K, rows, groups};
+    const cuuint64_t strides[2] = {K, K * rows};   // bytes, dims 1 and 2
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return FG_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lk(g_maps_mutex);
+        if (g_maps.size() > 512) g_maps.clear();
+        g_maps[key] = m;
+    }
+    *out = m;
+    return FG_OK;
+}
+
+// ---- configuration -----------------------------------------------------------
+// Cost model for one candidate block width, in SM clock cycles:
+//   per K block a tile needs max(MMA, shared-memory read, L2->SM load) cycles;
+//   MMA = 2*BN (8192 E4M3 MAC/clk/SM), shared-memory reads of the MMA =
+//   (16 KiB of A + 128*BN of B) / 128 B/clk, loads = (valid A rows*128 +
+//   128*BN) / 64 B/clk.  Tiles per CTA = ceil(tiles / grid).  The whole job is
+//   also bounded below by its unique HBM bytes at ~3.5 KB/clk.
+double estimate_cycles(int rows_per_block_valid, long long tiles, int KB, int BN, int grid, double hbm_bytes) {
+    const double mma = 2.0 * BN;
+    const double smem = (16384.0 + 128.0 * BN) / 128.0;
+    const double load = (rows_per_block_valid * 128.0 + 128.0 * BN) / 64.0;
+    const double per_kb = std::max(mma, std::max(smem, load));
+    const double waves = static_cast<double>((tiles + grid - 1) / grid);
+    const double epilogue = 2.0 * BN + 600.0;
+    const double t_tiles = waves * (KB * per_kb + epilogue);
+    const double t_hbm = hbm_bytes / 3500.0;
+    return std::max(t_tiles, t_hbm) + 2000.0;
+}
+
+int choose_block_n(long long rows_total_blocks, int valid_rows_per_block, int N, int K, int num_sms,
+                   double hbm_bytes) {
+    const char* force = std::getenv("FG_FORCE_BLOCK_N");
+    if (force) {
+        int f = std::atoi(force);
+        if (f >= 16 && f <= 256 && f % 16 == 0) return f;
+    }
+    const int KB = K / BK;
+    int best = 16;
+    double best_t = 1e300;
+    for (int bn = 16; bn <= 256; bn += 16) {
+        const long long tiles = rows_total_blocks * ((N + bn - 1) / bn);
+        const int grid = static_cast<int>(std::min<long long>(tiles, num_sms));
+        const double t = estimate_cycles(valid_rows_per_block, tiles, KB, bn, std::max(grid, 1), hbm_bytes);
+        if (t < best_t * 0.999 || (t <= best_t * 1.001 && bn > best)) {
+            if (t < best_t) best_t = t;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+int stage_bytes_for(int bn) { return BM * BK + bn * BK; }
+
+int choose_stages(int bn) {
+    const int sb = stage_bytes_for(bn);
+    int s = 8;
+    while (s > 2 && gemm_smem_bytes(sb, s) > static_cast<size_t>(kMaxDynamicSmem)) --s;
+    return s;
+}
+
+fg_status launch_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
+                    size_t smem, cudaStream_t st) {
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (bn) {
+#define FG8_CASE(BNV) \
+    case BNV:         \
+        e = launch_gemm<BNV>(ta, tb, p, grid, smem, st); \
+        break;
+        FG8_FOR_EACH_BN(FG8_CASE)
+#undef FG8_CASE
+        default:
+            return FG_ERR_UNSUPPORTED;
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return FG_ERR_CUDA;
+    }
+    return FG_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+constexpr long long kMaxDim = (1ll << 31) - 1;
+
+// Shared by the three GEMM kinds once their arguments are checked.
+fg_status run_gemm(int layout, const void* A, const float* sfa, const void* B, const float* sfb, void* D,
+                   const int* m_indices, const int* masked_m, int rows, int N, int K, int G, int valid_rows_hint,
+                   cudaStream_t stream) {
+    DeviceInfo* dev = nullptr;
+    fg_status st = current_device(&dev);
+    if (st != FG_OK) return st;
+    const int num_sms = effective_sms(*dev);
+    const int KB = K / BK;
+    const int NB = (N + 127) / 128;
+    const int a_groups = layout == LAYOUT_MASKED ? G : 1;
+    const long long m_blocks = (rows + BM - 1) / BM;
+    const long long row_blocks_total = m_blocks * a_groups;
+    const int valid_rows = std::min(BM, std::max(1, valid_rows_hint));
+    const double hbm = static_cast<double>(a_groups) * rows * K + static_cast<double>(G) * N * K +
+                       2.0 * a_groups * rows * N;
+    const int bn = choose_block_n(row_blocks_total, valid_rows, N, K, num_sms, hbm);
+    const int stages = choose_stages(bn);
+    const size_t smem = gemm_smem_bytes(stage_bytes_for(bn), stages);
+
+    CUtensorMap ta, tb;
+    st = operand_map(A, K, rows, a_groups, BM, &ta);
+    if (st != FG_OK) return st;
+    st = operand_map(B, K, N, G, bn, &tb);
+    if (st != FG_OK) return st;
+
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.layout = layout;
+    p.rows = rows;
+    p.N = N;
+    p.K = K;
+    p.G = G;
+    p.KB = KB;
+    p.NB = NB;
+    p.num_m_blocks = static_cast<int>(m_blocks);
+    p.num_n_blocks = (N + bn - 1) / bn;
+    p.raster_m = 16;
+    p.stages = stages;
+    p.sfa_ld = static_cast<int>(fg_get_tma_aligned_size(rows, 4));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.D = static_cast<__nv_bfloat16*>(D);
+    p.m_indices = m_indices;
+    p.masked_m = masked_m;
+    p.status = dev->status;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+
+    long long tiles = row_blocks_total * p.num_n_blocks;
+    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(tiles, num_sms)));
+    return launch_bn(bn, ta, tb, p, grid, smem, stream);
+}
+
+__global__ void sfa_transform_kernel(const float* __restrict__ in, float* __restrict__ out, int G, int M, int KB,
+                                     int M_pad) {
+    // One thread per output element, consecutive threads along m (coalesced stores).
+    const long long total = static_cast<long long>(G) * KB * M_pad;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int m = static_cast<int>(i % M_pad);
+        const long long gk = i / M_pad;
+        const int kb = static_cast<int>(gk % KB);
+        const int g = static_cast<int>(gk / KB);
+        out[i] = m < M ? in[(static_cast<long long>(g) * M + m) * KB + kb] : 0.0f;
+    }
+}
+
+struct EnvInit {
+    EnvInit() {
+        const char* w = std::getenv("FG_WAIT_LIMIT_NS");
+        if (w) {
+            unsigned long long v = std::strtoull(w, nullptr, 10);
+            if (v >= 1000) g_wait_limit_ns.store(v);
+        }
+    }
+} g_env_init;
+
+}  // namespace
+}  // namespace fg8
+
+using namespace fg8;
+
+extern "C" {
+
+const char* fg_status_string(int s) {
+    switch (s) {
+        case FG_OK: return "FG_OK";
+        case FG_ERR_INVALID_ARG: return "FG_ERR_INVALID_ARG";
+        case FG_ERR_ALIGNMENT: return "FG_ERR_ALIGNMENT";
+        case FG_ERR_UNSUPPORTED: return "FG_ERR_UNSUPPORTED";
+        case FG_ERR_NO_DEVICE: return "FG_ERR_NO_DEVICE";
+        case FG_ERR_CUDA: return "FG_ERR_CUDA";
+        case FG_ERR_TIMEOUT: return "FG_ERR_TIMEOUT";
+        default: return "FG_ERR_UNKNOWN";
+    }
+}
+
+const char* fg_version(void) { return "fg8 0.1.0 sm_100a"; }
+
+fg_status fg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* D, int M, int N,
+                         int K, fg_stream_t stream) {
+    if (M < 0 || N < 0 || K < 0) return FG_ERR_INVALID_ARG;
+    if (K == 0 || K % 128 != 0 || N % 16 != 0) return FG_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return FG_OK;
+    if (!A || !sfa || !B || !sfb || !D) return FG_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sfa) || !aligned4(sfb))
+        return FG_ERR_ALIGNMENT;
+    if (static_cast<long long>(M) * N > kMaxDim * 4 || M > kMaxDim - 128) return FG_ERR_UNSUPPORTED;
+    return run_gemm(LAYOUT_NORMAL, A, sfa, B, sfb, D, nullptr, nullptr, M, N, K, 1, M,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+fg_status fg_m_grouped_fp8_gemm_nt_contiguous(const void* A, const float* sfa, const void* B, const float* sfb,
+                                              void* D, const int* m_indices, int M_tot, int N, int K, int G,
+                                              fg_stream_t stream) {
+    if (M_tot < 0 || N < 0 || K < 0 || G <= 0) return FG_ERR_INVALID_ARG;
+    if (K == 0 || K % 128 != 0 || N % 16 != 0) return FG_ERR_UNSUPPORTED;
+    if (M_tot % fg_get_m_alignment_for_contiguous_layout() != 0) return FG_ERR_INVALID_ARG;
+    if (M_tot == 0 || N == 0) return FG_OK;
+    if (!A || !sfa || !B || !sfb || !D || !m_indices) return FG_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sfa) || !aligned4(sfb) ||
+        !aligned4(m_indices))
+        return FG_ERR_ALIGNMENT;
+    if (M_tot > kMaxDim - 128) return FG_ERR_UNSUPPORTED;
+    return run_gemm(LAYOUT_CONTIGUOUS, A, sfa, B, sfb, D, m_indices, nullptr, M_tot, N, K, G, BM,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+fg_status fg_m_grouped_fp8_gemm_nt_masked(const void* A, const float* sfa, const void* B, const float* sfb,
+                                          void* D, const int* masked_m, int G, int M_max, int N, int K,
+                                          int expected_m, fg_stream_t stream) {
+    if (G < 0 || M_max < 0 || N < 0 || K < 0 || expected_m < 0) return FG_ERR_INVALID_ARG;
+    if (K == 0 || K % 128 != 0 || N % 16 != 0) return FG_ERR_UNSUPPORTED;
+    if (G == 0 || M_max == 0 || N == 0) return FG_OK;
+    if (!A || !sfa || !B || !sfb || !D || !masked_m) return FG_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sfa) || !aligned4(sfb) ||
+        !aligned4(masked_m))
+        return FG_ERR_ALIGNMENT;
+    if (static_cast<long long>(G) * M_max > kMaxDim - 128) return FG_ERR_UNSUPPORTED;
+    const int hint = expected_m > 0 ? std::min(expected_m, M_max) : M_max;
+    return run_gemm(LAYOUT_MASKED, A, sfa, B, sfb, D, nullptr, masked_m, M_max, N, K, G, hint,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fg_get_num_sms(void) {
+    const int n = g_num_sms.load();
+    if (n > 0) return n;
+    DeviceInfo* d = nullptr;
+    if (current_device(&d) != FG_OK) {
+        const char* env = std::getenv("FG_NUM_SMS");
+        return env ? std::max(0, std::atoi(env)) : 0;
+    }
+    return effective_sms(*d);
+}
+
+fg_status fg_set_num_sms(int n) {
+    if (n <= 0) return FG_ERR_INVALID_ARG;
+    DeviceInfo* d = nullptr;
+    const fg_status st = current_device(&d);
+    if (st == FG_OK && n > d->sm_count) return FG_ERR_INVALID_ARG;
+    g_num_sms.store(n);
+    return FG_OK;
+}
+
+int fg_get_m_alignment_for_contiguous_layout(void) { return BM; }
+
+size_t fg_get_tma_aligned_size(size_t n, size_t elem_bytes) {
+    if (elem_bytes == 0 || 16 % elem_bytes != 0) return 0;
+    const size_t a = 16 / elem_bytes;
+    return (n + a - 1) / a * a;
+}
+
+fg_status fg_transform_sfa_to_tma_layout(const float* in, float* out, int G, int M, int KB, fg_stream_t stream) {
+    if (G < 0 || M < 0 || KB < 0) return FG_ERR_INVALID_ARG;
+    if (G == 0 || M == 0 || KB == 0) return FG_OK;
+    if (!in || !out) return FG_ERR_INVALID_ARG;
+    if (!aligned4(in) || !aligned16(out)) return FG_ERR_ALIGNMENT;
+    DeviceInfo* d = nullptr;
+    fg_status st = current_device(&d);
+    if (st != FG_OK) return st;
+    const int M_pad = static_cast<int>(fg_get_tma_aligned_size(M, 4));
+    const long long total = static_cast<long long>(G) * KB * M_pad;
+    const int threads = 256;
+    const long long blocks = std::min<long long>((total + threads - 1) / threads, 8LL * d->sm_count);
+    sfa_transform_kernel<<<static_cast<int>(blocks), threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        in, out, G, M, KB, M_pad);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FG_OK : FG_ERR_CUDA;
+}
+
+fg_status fg_get_last_device_status(fg_stream_t stream, int* code_out, int* detail_out) {
+    if (!code_out) return FG_ERR_INVALID_ARG;
+    DeviceInfo* d = nullptr;
+    fg_status st = current_device(&d);
+    if (st != FG_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return FG_ERR_CUDA;
+    }
+    int h[2] = {0, 0};
+    const int zero[2] = {0, 0};
+    if (cudaMemcpyFromSymbol(h, g_status, sizeof(h)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_status, zero, sizeof(zero)) != cudaSuccess) {
+        cudaGetLastError();
+        return FG_ERR_CUDA;
+    }
+    *code_out = h[0];
+    if (detail_out) *detail_out = h[1];
+    return FG_OK;
+}
+
+fg_status fg_set_wait_limit_ns(unsigned long long ns) {
+    if (ns < 1000) return FG_ERR_INVALID_ARG;
+    g_wait_limit_ns.store(ns);
+    return FG_OK;
+}
+
+unsigned long long fg_get_wait_limit_ns(void) { return g_wait_limit_ns.load(); }
+
+int fg_query_block_n(int M, int N, int K) {
+    if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0 || N % 16 != 0) return 0;
+    DeviceInfo* d = nullptr;
+    int sms = 148;
+    if (current_device(&d) == FG_OK) sms = effective_sms(*d);
+    else if (g_num_sms.load() > 0) sms = g_num_sms.load();
+    const double hbm = static_cast<double>(M) * K + static_cast<double>(N) * K + 2.0 * M * N;
+    return choose_block_n((M + BM - 1) / BM, std::min(M, BM), N, K, sms, hbm);
+}
+
+}  // extern "C"

@@ -1,0 +1,164 @@
+/*
+ * fg8.h -- C ABI of libfg8.so: fine-grained-scaled FP8 GEMM for NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation (fine-grained scaling "as proposed in DeepSeek-V3":
+ * chujupifa.com "机器之心报道", opening summary; deepseek.csdn.net
+ * "DeepGEMM：简洁、高效，用约300行CUDA代码重构AI计算的底层法则", section
+ * "什么是DeepGEMM呢？"):
+ *
+ *   D[m,n] = bf16( sum_kb ( sum_{k in kb} A[m,k] * B[n,k] ) * sfa[m,kb] * sfb[n/128,kb] )
+ *
+ * with kb running over 128-wide blocks of K, A and B stored as E4M3 codes
+ * (4 exponent bits, 3 mantissa bits: ai.abqq.net "DeepSeek开源周第三天…
+ * DeepGEMM：FP8", section 3 "核心功能与特性"; OCP E4M3 "FN": max 448, no
+ * infinities), one FP32 scale per 1x128 block of A (sfa) and per 128x128
+ * block of B (sfb), and the result rounded to BF16 (round to nearest even).
+ * "NT": both operands are K-major (row-major A [M,K] and B [N,K]).
+ *
+ * Three GEMM kinds are provided, the ones the pages list (ai.abqq.net section
+ * 3; game.3loumao.org explainer, section "03 DeepSeek是如何创新的？"): normal,
+ * contiguous-grouped MoE and masked-grouped MoE.  The helper functions mirror
+ * the utilities of the csdn page, section "实用工具".
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees or retains them beyond the call (a small cache of TMA
+ *    descriptors is keyed by pointer and shape).
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream) and never
+ *    synchronise.  Errors detectable on the host are returned before anything
+ *    is launched, and then D is untouched.
+ *  - Errors detected on the device (a pipeline wait that timed out) are
+ *    recorded in a per-device status word read by fg_get_last_device_status.
+ *  - E4M3 operands: 1 byte per element.  Scales: IEEE fp32.  D: bf16.
+ *  - Pointer alignment: A, B, D, sfa 16 bytes; sfb 4 bytes.
+ *  - K must be a positive multiple of 128; N a positive multiple of 16.
+ */
+#ifndef FG8_H
+#define FG8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fg_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    FG_OK = 0,
+    FG_ERR_INVALID_ARG = 1, /* null pointer, negative or inconsistent size */
+    FG_ERR_ALIGNMENT = 2,   /* a pointer breaks the 16-byte rule above */
+    FG_ERR_UNSUPPORTED = 3, /* K % 128 != 0, N % 16 != 0, size beyond limits */
+    FG_ERR_NO_DEVICE = 4,   /* no CUDA device, or not an sm_100 device */
+    FG_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed */
+    FG_ERR_TIMEOUT = 6      /* device side: a pipeline wait ran past its limit */
+} fg_status;
+
+/* Human-readable name of a status code (static string). */
+const char* fg_status_string(int status);
+
+/* Library version, e.g. "fg8 0.1.0 sm_100a". */
+const char* fg_version(void);
+
+/*
+ * Normal GEMM, D = A . B^T with fine-grained scales.
+ *   A   [M, K]   E4M3, row-major (row stride K bytes)
+ *   sfa [K/128][M_pad] fp32: MN-major ("column-major, TMA-aligned") scales of
+ *       A, M_pad = fg_get_tma_aligned_size(M, 4); sfa[kb*M_pad + m] scales
+ *       A[m, 128*kb .. 128*kb+127].  Build it with fg_transform_sfa_to_tma_layout.
+ *   B   [N, K]   E4M3, row-major
+ *   sfb [ceil(N/128)][K/128] fp32 row-major: sfb[nb*(K/128) + kb] scales
+ *       B[128*nb .. 128*nb+127, 128*kb .. 128*kb+127]
+ *   D   [M, N]   bf16, row-major (row stride N elements), fully overwritten
+ * M == 0 is a no-op.  Returns FG_OK or an error code.
+ */
+fg_status fg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* D, int M,
+                         int N, int K, fg_stream_t stream);
+
+/*
+ * Contiguous-grouped MoE GEMM (game.3loumao.org explainer section 03: the
+ * rows of all experts "joined into one block").  Each expert's rows form one
+ * segment of A; every segment is padded up to a multiple of
+ * fg_get_m_alignment_for_contiguous_layout() rows and the segments are
+ * concatenated along M.
+ *   A         [M_tot, K] E4M3;   sfa [K/128][M_pad(M_tot)] MN-major
+ *   B         [G, N, K]  E4M3;   sfb [G][ceil(N/128)][K/128]
+ *   m_indices [M_tot] int32 (device): the expert of each row, or -1 on padding
+ *   D         [M_tot, N] bf16
+ * Row m of D is written iff 0 <= m_indices[m] < G, with
+ *   D[m,:] = GEMM(A[m,:], B[m_indices[m]], sfb[m_indices[m]]).
+ * Rows tagged -1 are never written.  Preconditions checked on the host:
+ * M_tot % alignment == 0.  Preconditions NOT checked (device data): all rows
+ * of one aligned block carry the same expert or -1, and a block's first row
+ * is not -1 unless the whole block is padding; rows that break this are left
+ * unwritten.
+ */
+fg_status fg_m_grouped_fp8_gemm_nt_contiguous(const void* A, const float* sfa, const void* B,
+                                              const float* sfb, void* D, const int* m_indices, int M_tot,
+                                              int N, int K, int G, fg_stream_t stream);
+
+/*
+ * Masked-grouped MoE GEMM (game.3loumao.org explainer section 03: a mask
+ * marks which rows to compute; empty rows are skipped).
+ *   A        [G, M_max, K] E4M3;  sfa [G][K/128][M_pad(M_max)] MN-major
+ *   B        [G, N, K]     E4M3;  sfb [G][ceil(N/128)][K/128]
+ *   masked_m [G] int32 (device): rows r < min(masked_m[g], M_max) of group g
+ *            are computed; the other rows of D[g] are never written, and a
+ *            group with masked_m[g] <= 0 costs nothing (its B is not read).
+ *   D        [G, M_max, N] bf16
+ *   expected_m: host-side hint of the typical masked_m used to pick the tile
+ *            shape (0 = M_max).  It never changes the result.
+ */
+fg_status fg_m_grouped_fp8_gemm_nt_masked(const void* A, const float* sfa, const void* B, const float* sfb,
+                                          void* D, const int* masked_m, int G, int M_max, int N, int K,
+                                          int expected_m, fg_stream_t stream);
+
+/* Maximum number of SMs the GEMM kernels use (csdn page, "实用工具":
+ * set_num_sms / get_num_sms).  Process-global.  Default: the device's SM
+ * count (or the FG_NUM_SMS environment variable).  fg_set_num_sms accepts
+ * 1 .. device SM count and returns FG_ERR_INVALID_ARG otherwise. */
+int fg_get_num_sms(void);
+fg_status fg_set_num_sms(int n);
+
+/* Row alignment of each expert segment in the contiguous layout (csdn page,
+ * "实用工具": get_m_alignment_for_contiguous_layout).  Returns 128, the row
+ * block of the kernels. */
+int fg_get_m_alignment_for_contiguous_layout(void);
+
+/* Smallest n' >= n with n' * elem_bytes a multiple of 16 bytes, the TMA
+ * stride rule (csdn page, "实用工具": get_tma_aligned_size).  elem_bytes must
+ * divide 16; returns 0 otherwise. */
+size_t fg_get_tma_aligned_size(size_t n, size_t elem_bytes);
+
+/* Scale layout transform (csdn page, "实用工具": get_col_major_tma_aligned_tensor).
+ *   in  [G][M][KB] fp32 row-major (device)
+ *   out [G][KB][M_pad] fp32 (device), M_pad = fg_get_tma_aligned_size(M, 4):
+ *       out[g][kb][m] = in[g][m][kb] for m < M, 0 for M <= m < M_pad.
+ * Both pointers 16-byte aligned (in: 4).  Runs one small kernel on stream. */
+fg_status fg_transform_sfa_to_tma_layout(const float* in, float* out, int G, int M, int KB, fg_stream_t stream);
+
+/* Reads and clears this device's status word after synchronising `stream`.
+ * *code_out = 0 when no kernel recorded an error since the last call, else
+ * FG_ERR_TIMEOUT; *detail_out (may be NULL) = (block << 8) | role of the
+ * first failure (role 1 = TMA producer, 2 = MMA issuer, 3 = epilogue). */
+fg_status fg_get_last_device_status(fg_stream_t stream, int* code_out, int* detail_out);
+
+/* Upper bound, in nanoseconds, on any single pipeline wait inside the GEMM
+ * kernels (default 1e9 = 1 s; FG_WAIT_LIMIT_NS overrides at load).  A wait
+ * that runs past it makes the kernel record FG_ERR_TIMEOUT, drain its copies
+ * in flight, release tensor memory and return: it never hangs the GPU.
+ * Values below 1000 are rejected. */
+fg_status fg_set_wait_limit_ns(unsigned long long ns);
+unsigned long long fg_get_wait_limit_ns(void);
+
+/* The block width (BLOCK_N) the normal GEMM would use for (M, N, K) with the
+ * current SM budget, or 0 for an unsupported shape.  Diagnostics. */
+int fg_query_block_n(int M, int N, int K);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FG8_H */

@@ -1,0 +1,307 @@
+"""GPU parity: the CUDA path (through the C ABI binding) against the CPU oracle.
+
+Tolerance (per tensor, over written rows, in FP64):
+    1 - 2 sum(xy) / sum(x^2 + y^2) <= 1e-3   and   max|x - y| <= 1e-2 * max|y|.
+Rows the GEMM must not write (padding rows tagged -1, rows past masked_m) are
+pre-filled with a sentinel and must come back bit-identical.  Cases whose
+exact result is representable in BF16 (permutation B, small integers) must be
+bit-exact.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+DIFF_TOL = 1e-3
+MAX_TOL = 1e-2
+SENTINEL = -12345.0  # exactly representable in bf16 (0xC640 pattern after rounding is fixed below)
+
+
+@pytest.fixture(scope="module")
+def fg():
+    import fp8_fine_grained_tma_b200 as fg
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return fg
+
+
+@pytest.fixture(autouse=True)
+def clean_status(fg):
+    fg.get_last_device_status()
+    yield
+    code, detail = fg.get_last_device_status()
+    assert code == 0, f"device status {code} detail {detail:#x}"
+
+
+def check(gpu_rows: np.ndarray, ref_rows: np.ndarray):
+    c = oracle.compare(gpu_rows, ref_rows)
+    assert np.all(np.isfinite(gpu_rows))
+    assert c["diff"] <= DIFF_TOL, c
+    assert c["rel_max_err"] <= MAX_TOL, c
+    return c
+
+
+def bf16_of(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16)
+
+
+def sentinel_bf16():
+    return torch.tensor(SENTINEL, dtype=torch.bfloat16)
+
+
+def to_gpu_normal(fg, x):
+    A = x.A.cuda()
+    B = x.B.cuda()
+    sfa = fg.get_col_major_tma_aligned_tensor(x.sfa.cuda())
+    sfb = x.sfb.cuda()
+    return A, sfa, B, sfb
+
+
+# --------------------------------------------------------------- helpers --
+
+def test_sfa_transform_matches_oracle(fg):
+    g = torch.Generator().manual_seed(5)
+    for G, M, KB in [(1, 37, 5), (3, 256, 56), (2, 1, 1), (1, 4096, 12)]:
+        s = torch.randn((G, M, KB), generator=g)
+        out = fg.get_col_major_tma_aligned_tensor(s.cuda())
+        m_pad = fg.get_tma_aligned_size(M, 4)
+        storage = torch.as_strided(out, (G, KB, m_pad), (KB * m_pad, m_pad, 1)).cpu().numpy()
+        assert np.array_equal(storage, oracle.sfa_to_mn_major(s.numpy()))
+        assert torch.equal(out.cpu(), s)
+
+
+# ----------------------------------------------------------- normal GEMM --
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 128), (1, 16, 128), (200, 272, 512), (257, 2112, 1024),
+                                   (64, 2112, 7168), (383, 4096, 256)])
+def test_normal_gemm_matches_oracle(fg, M, N, K):
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(0, 50) + M + N)
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    D = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    check(D.double().cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("bn", list(range(16, 257, 16)))
+def test_every_block_width_matches_oracle(fg, bn, monkeypatch):
+    monkeypatch.setenv("FG_FORCE_BLOCK_N", str(bn))
+    M, N, K = 300, 400, 384   # ragged M and N, several K blocks, tiles straddling scale blocks
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(0, 60) + bn)
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    D = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    check(D.double().cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("bn", [16, 112, 256])
+def test_permutation_b_is_bit_exact(fg, bn, monkeypatch):
+    monkeypatch.setenv("FG_FORCE_BLOCK_N", str(bn))
+    M, K = 130, 384
+    N = K
+    rng = np.random.default_rng(3)
+    perm = rng.permutation(K)
+    g = torch.Generator().manual_seed(3)
+    A = synth.random_codes((M, K), g).numpy()
+    B = np.zeros((N, K), dtype=np.uint8)
+    B[np.arange(N), perm] = 0x38
+    sfa = (2.0 ** rng.integers(-3, 4, (M, K // 128))).astype(np.float32)
+    sfb = np.ones((N // 128, K // 128), dtype=np.float32)
+    ref = oracle.gemm_nt(A, sfa, B, sfb)
+    D = fg.fp8_gemm_nt(torch.from_numpy(A).cuda(), fg.get_col_major_tma_aligned_tensor(torch.from_numpy(sfa).cuda()),
+                       torch.from_numpy(B).cuda(), torch.from_numpy(sfb).cuda())
+    assert torch.equal(D.cpu().view(torch.int16), bf16_of(ref).view(torch.int16))
+
+
+def test_integer_inputs_are_bit_exact(fg):
+    M, N, K = 256, 320, 256
+    rng = np.random.default_rng(4)
+    code = {-1: 0xB8, 0: 0x00, 1: 0x38}
+    Ai = rng.choice([-1, 0, 1], (M, K))
+    Bi = rng.choice([-1, 0, 1], (N, K))
+    A = np.vectorize(code.get)(Ai).astype(np.uint8)
+    B = np.vectorize(code.get)(Bi).astype(np.uint8)
+    sfa = np.ones((M, K // 128), np.float32)
+    sfb = np.ones(((N + 127) // 128, K // 128), np.float32)
+    expect = (Ai @ Bi.T).astype(np.float64)
+    assert np.abs(expect).max() <= 256
+    D = fg.fp8_gemm_nt(torch.from_numpy(A).cuda(), fg.get_col_major_tma_aligned_tensor(torch.from_numpy(sfa).cuda()),
+                       torch.from_numpy(B).cuda(), torch.from_numpy(sfb).cuda())
+    assert torch.equal(D.cpu().view(torch.int16), bf16_of(expect).view(torch.int16))
+
+
+def test_repeated_launches_on_a_side_stream(fg):
+    x = synth.normal_inputs(256, 512, 1024, seed=synth.seed_for(0, 70))
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    s = torch.cuda.Stream()
+    outs = []
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            outs.append(fg.fp8_gemm_nt(A, sfa, B, sfb))
+    s.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    check(outs[0].double().cpu().numpy(), ref)
+
+
+def test_num_sms_limit_keeps_results(fg):
+    x = synth.normal_inputs(512, 1024, 512, seed=synth.seed_for(0, 71))
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    full = fg.get_num_sms()
+    D0 = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    try:
+        fg.set_num_sms(7)
+        assert fg.get_num_sms() == 7
+        D1 = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    finally:
+        fg.set_num_sms(full)
+    assert torch.equal(D0, D1)
+
+
+# ----------------------------------------------------------- grouped GEMMs --
+
+def run_contiguous(fg, x):
+    A = x.A.cuda()
+    sfa = fg.get_col_major_tma_aligned_tensor(x.sfa.cuda())
+    D = torch.full((x.M_tot, x.N), SENTINEL, dtype=torch.bfloat16, device="cuda")
+    fg.m_grouped_fp8_gemm_nt_contiguous(A, sfa, x.B.cuda(), x.sfb.cuda(), x.m_indices.cuda(), D=D)
+    torch.cuda.synchronize()
+    return D
+
+
+def check_contiguous(fg, x, D, rows=None):
+    mi = x.m_indices.numpy()
+    pad = mi < 0
+    Dc = D.cpu()
+    assert torch.all(Dc[torch.from_numpy(pad)].view(torch.int16) == sentinel_bf16().view(torch.int16))
+    if rows is None:
+        rows = np.nonzero(~pad)[0]
+    ref, written = oracle.m_grouped_contiguous(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), mi,
+                                               rows=rows)
+    assert written.all()
+    check(Dc[torch.from_numpy(np.asarray(rows))].double().numpy(), ref)
+
+
+def test_contiguous_small(fg):
+    x = synth.contiguous_inputs(4, 272, 512, seed=synth.seed_for(2, 50), counts=[5, 0, 130, 256])
+    D = run_contiguous(fg, x)
+    check_contiguous(fg, x, D)
+
+
+def test_contiguous_all_padding_block_is_skipped(fg):
+    x = synth.contiguous_inputs(2, 128, 256, seed=synth.seed_for(2, 51), counts=[100, 40])
+    # add an all-padding block between the experts
+    mi = x.m_indices.numpy()
+    A = torch.cat([x.A[:128], torch.zeros((128, 256), dtype=torch.uint8), x.A[128:]])
+    sfa = torch.cat([x.sfa[:128], torch.ones((128, 2)), x.sfa[128:]])
+    tags = np.concatenate([mi[:128], np.full(128, -1, np.int32), mi[128:]])
+    y = synth.ContiguousInputs(A, sfa, x.B, x.sfb, torch.from_numpy(tags), x.counts, 2, 128, 256)
+    D = run_contiguous(fg, y)
+    check_contiguous(fg, y, D)
+
+
+def run_masked(fg, x, expected_m=0):
+    sfa = fg.get_col_major_tma_aligned_tensor(x.sfa.cuda())
+    D = torch.full((x.G, x.M_max, x.N), SENTINEL, dtype=torch.bfloat16, device="cuda")
+    fg.m_grouped_fp8_gemm_nt_masked(x.A.cuda(), sfa, x.B.cuda(), x.sfb.cuda(), x.masked_m.cuda(),
+                                    expected_m=expected_m, D=D)
+    torch.cuda.synchronize()
+    return D
+
+
+def check_masked(fg, x, D, sample=None):
+    mm = x.masked_m.numpy()
+    Dc = D.cpu()
+    lim = np.minimum(np.maximum(mm, 0), x.M_max)
+    written = np.arange(x.M_max)[None, :] < lim[:, None]
+    flat = Dc.view(-1, x.N)
+    unw = torch.from_numpy(~written.reshape(-1))
+    assert torch.all(flat[unw].view(torch.int16) == sentinel_bf16().view(torch.int16))
+    rows = np.nonzero(written.reshape(-1))[0]
+    if sample is not None and len(rows) > sample:
+        rng = np.random.default_rng(0)
+        rows = np.sort(rng.choice(rows, sample, replace=False))
+    if len(rows) == 0:
+        return
+    ref, w = oracle.m_grouped_masked(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), mm, rows=rows)
+    assert w.all()
+    check(flat[torch.from_numpy(rows)].double().numpy(), ref)
+
+
+def test_masked_small(fg):
+    x = synth.masked_inputs(5, 200, 144, 384, seed=synth.seed_for(3, 50), masked=[0, 1, 128, 200, 250])
+    D = run_masked(fg, x)
+    check_masked(fg, x, D)
+
+
+def test_masked_all_empty(fg):
+    x = synth.masked_inputs(3, 64, 64, 128, seed=synth.seed_for(3, 51), masked=[0, 0, -5])
+    D = run_masked(fg, x)
+    check_masked(fg, x, D)
+
+
+# ------------------------------------------- the workloads, at full size --
+
+def sample_rows(M, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = set([0, M - 1, min(M - 1, 127), min(M - 1, 128)])
+    rows |= set(int(r) for r in rng.integers(0, M, n))
+    return np.array(sorted(rows))
+
+
+def test_decode_config_full(fg):
+    x = synth.normal_inputs(64, 2112, 7168, seed=synth.seed_for(0, 0))
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    D = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    check(D.double().cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("si,N,K", [(0, 24576, 1536), (1, 7168, 16384), (2, 4096, 7168)])
+def test_prefill_config_sampled_rows(fg, si, N, K):
+    M = 4096
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(1, si))
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    D = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    rows = sample_rows(M, 24, si)
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), rows=rows)
+    check(D[torch.from_numpy(rows).cuda()].double().cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("si,N,K", [(0, 4096, 7168), (1, 7168, 2048)])
+def test_contiguous_config_sampled_rows(fg, si, N, K):
+    x = synth.contiguous_inputs(8, N, K, seed=synth.seed_for(2, si))
+    D = run_contiguous(fg, x)
+    real = np.nonzero(x.m_indices.numpy() >= 0)[0]
+    rng = np.random.default_rng(si)
+    rows = np.sort(rng.choice(real, 32, replace=False))
+    check_contiguous(fg, x, D, rows=rows)
+
+
+@pytest.mark.parametrize("si,N,K", [(0, 4096, 7168), (1, 7168, 2048)])
+def test_masked_config_sampled_rows(fg, si, N, K):
+    x = synth.masked_inputs(32, 256, N, K, seed=synth.seed_for(3, si))
+    D = run_masked(fg, x, expected_m=128)
+    check_masked(fg, x, D, sample=32)
+
+
+@pytest.mark.parametrize("si,M,N,K", [(i * 2 + j, M, N, K) for j, M in enumerate([64, 128])
+                                      for i, (N, K) in enumerate([(2112, 7168), (24576, 1536), (32768, 512),
+                                                                  (7168, 16384), (4096, 7168), (7168, 2048)])])
+def test_decode_sweep_sampled_rows(fg, si, M, N, K):
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(4, si))
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    D = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    rows = sample_rows(M, 8, si)
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), rows=rows)
+    check(D[torch.from_numpy(rows).cuda()].double().cpu().numpy(), ref)
