@@ -13,7 +13,7 @@
 #include <mutex>
 #include <tuple>
 
-#include "../../include/fg8.h"
+#include "fg8.h"
 #include "launch.cuh"
 
 namespace fg8 {

@@ -13,7 +13,7 @@
 //   warp 8     TMA producer: one lane streams A [128 x 128] and B [BN x 128]
 //              E4M3 tiles into an S-stage shared-memory ring (128-byte swizzle).
 //   warp 9     MMA issuer: one lane issues 4 x tcgen05.mma kind::f8f6f4
-//              (M=128, N=BN, K=32) per K block into one of two TMEM
+//              (M=128, N=BN, K=32) per K block into one of NBUF (2..4) TMEM
 //              accumulators, overwriting it at the block's first MMA.
 //   warps 0-7  promotion + epilogue: two warpgroups split the tile's 16-column
 //              chunks; each thread owns one TMEM lane (= one output row), reads
@@ -39,7 +39,17 @@ constexpr int BK = 128;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
-constexpr int NUM_THREADS = 320;                   // 8 promotion warps + producer + MMA issuer
+constexpr int NUM_THREADS = 384;                   // 3 warpgroups: 2 promotion, 1 producer/MMA
+// Register split (setmaxnreg, inside each role's own branch): every thread is
+// launched with REGS_LAUNCH registers; the producer warpgroup (warps 8..11)
+// drops to REGS_PRODUCER and the two promotion warpgroups rise to
+// REGS_PROMOTION.  256 * 224 + 128 * 56 == 384 * 168, so the raise only uses
+// registers the block already owns.  The host launches a build only if its
+// register count is exactly REGS_LAUNCH (otherwise the raise could wait forever).
+constexpr int REGS_LAUNCH = 168;
+constexpr int REGS_PRODUCER = 56;
+constexpr int REGS_PROMOTION = 224;
+static_assert(256 * REGS_PROMOTION + 128 * REGS_PRODUCER <= NUM_THREADS * REGS_LAUNCH, "register split");
 constexpr int EPI_COLS = 32;                       // columns per staged piece
 constexpr int EPI_PITCH = EPI_COLS * 2 + 16;       // bytes per staged row (padding kills bank conflicts)
 constexpr int EPI_WARP_BYTES = 32 * EPI_PITCH;     // staging bytes per epilogue warp
@@ -78,19 +88,25 @@ struct GemmShape {
     static constexpr int B_TILE_BYTES = BN * BK;
     static constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
     static constexpr int ACC_STRIDE = (BN + 31) / 32 * 32;   // TMEM columns per accumulator
-    static constexpr int TMEM_COLS = 2 * ACC_STRIDE <= 32    ? 32
-                                     : 2 * ACC_STRIDE <= 64  ? 64
-                                     : 2 * ACC_STRIDE <= 128 ? 128
-                                     : 2 * ACC_STRIDE <= 256 ? 256
-                                                             : 512;
+    // As many K-block accumulators as TMEM holds (at most 4): the MMA issuer may
+    // run NBUF - 1 blocks ahead of the promotion warps.
+    static constexpr int NBUF = (512 / ACC_STRIDE) < 4 ? (512 / ACC_STRIDE) : 4;
+    static constexpr int TMEM_USED = NBUF * ACC_STRIDE;
+    static constexpr int TMEM_COLS = TMEM_USED <= 32    ? 32
+                                     : TMEM_USED <= 64  ? 64
+                                     : TMEM_USED <= 128 ? 128
+                                     : TMEM_USED <= 256 ? 256
+                                                        : 512;
+    static_assert(NBUF >= 2, "need two accumulators");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN must be a multiple of 16 in [16, 256]");
 };
 
 // Dynamic shared memory layout (after aligning the base to 1024 bytes):
 //   [stages x (A tile | B tile)] [8 x epilogue staging] [barriers] [tmem slot, abort flag]
+constexpr int MAX_NBUF = 4;
 __host__ __device__ constexpr size_t gemm_smem_bytes(int stage_bytes, int stages) {
     return 1024 + static_cast<size_t>(stages) * stage_bytes + NUM_EPI_WARPS * EPI_WARP_BYTES +
-           (2 * stages + 5) * 8 + 16;
+           (2 * stages + 2 * MAX_NBUF + 1) * 8 + 16;
 }
 
 struct TileInfo {
@@ -183,6 +199,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     using S = GemmShape<BN>;
     constexpr int NC = S::NC;
     constexpr int CPW = S::CPW;
+    constexpr int LB = CPW <= 4 ? CPW : 4;   // chunks read from TMEM per wait
     constexpr uint32_t IDESC = ptx::idesc_e4m3_f32(BM, BN);
 
     extern __shared__ uint8_t smem_raw[];
@@ -192,8 +209,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(epi_base + NUM_EPI_WARPS * EPI_WARP_BYTES);
     uint64_t* empty = full + p.stages;
     uint64_t* tfull = empty + p.stages;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* done_bar = tempty + 2;
+    uint64_t* tempty = tfull + S::NBUF;
+    uint64_t* done_bar = tempty + S::NBUF;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -207,7 +224,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < S::NBUF; ++b) {
             ptx::mbar_init(&tfull[b], 1);
             ptx::mbar_init(&tempty[b], NUM_EPI_WARPS);
         }
@@ -226,7 +243,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == PRODUCER_WARP) {
+    if (warp >= NUM_EPI_WARPS) {
+      ptx::setmaxnreg_dec<REGS_PRODUCER>();
+      if (warp == PRODUCER_WARP) {
         if (lane == 0) {
             TileScheduler sch;
             TileInfo t;
@@ -272,7 +291,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             }
         }
-    } else if (warp == MMA_WARP) {
+      } else if (warp == MMA_WARP) {
         if (lane == 0) {
             TileScheduler sch;
             TileInfo t;
@@ -305,8 +324,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         stage = 0;
                         phase ^= 1u;
                     }
-                    buf ^= 1;
-                    if (buf == 0) bphase ^= 1u;
+                    if (++buf == S::NBUF) {
+                        buf = 0;
+                        bphase ^= 1u;
+                    }
                 }
             }
             if (w == 2) record_error(p.status, ERR_TIMEOUT, ROLE_MMA);
@@ -314,7 +335,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::mma_commit(done_bar);
             ptx::mbar_wait(done_bar, 0, drain_limit);
         }
-    } else if (warp < NUM_EPI_WARPS) {
+      }
+    } else {
+        ptx::setmaxnreg_inc<REGS_PROMOTION>();
         // ---- promotion + epilogue: warps 0..7 ----
         const int wg = warp / 4;
         const int quarter = warp % 4;                 // TMEM lanes 32*quarter .. +31
@@ -368,34 +391,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 ptx::tc_fence_after();
                 const uint32_t tbase = tmem_base + lane_base + static_cast<uint32_t>(buf * S::ACC_STRIDE);
+                // Read the block's partial sums in batches of LB chunks (one
+                // tcgen05.wait::ld per batch), then scale and accumulate.
 #pragma unroll
-                for (int i = 0; i < CPW; i += 2) {
-                    const int c0 = chunk0 + i;
-                    const bool has0 = c0 < NC;
-                    const bool has1 = (i + 1 < CPW) && (c0 + 1 < NC);
-                    uint32_t r0[16], r1[16];
-                    if (has0) ptx::tmem_ld16(tbase + static_cast<uint32_t>(c0 * 16), r0);
-                    if (has1) ptx::tmem_ld16(tbase + static_cast<uint32_t>((c0 + 1) * 16), r1);
-                    if (i + 1 < CPW) ptx::tmem_wait_ld(r0, r1);
-                    else ptx::tmem_wait_ld(r0);
-                    if (has0) {
-                        const float s = (n0 + c0 * 16 >= split_col) ? s_hi : s_lo;
+                for (int i0 = 0; i0 < CPW; i0 += LB) {
+                    uint32_t r[LB][16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) acc[i][j] = fmaf(__uint_as_float(r0[j]), s, acc[i][j]);
+                    for (int b = 0; b < LB; ++b) {
+                        const int c = chunk0 + i0 + b;
+                        if (i0 + b < CPW && c < NC) ptx::tmem_ld16(tbase + static_cast<uint32_t>(c * 16), r[b]);
                     }
-                    if (has1) {
-                        const float s = (n0 + (c0 + 1) * 16 >= split_col) ? s_hi : s_lo;
+                    ptx::tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            acc[(i + 1) < CPW ? i + 1 : i][j] =
-                                fmaf(__uint_as_float(r1[j]), s, acc[(i + 1) < CPW ? i + 1 : i][j]);
+                    for (int b = 0; b < LB; ++b) ptx::reg_fence(r[b]);
+#pragma unroll
+                    for (int b = 0; b < LB; ++b) {
+                        const int i = i0 + b;
+                        const int c = chunk0 + i;
+                        if (i < CPW && c < NC) {
+                            const float sc = (n0 + c * 16 >= split_col) ? s_hi : s_lo;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                acc[i < CPW ? i : 0][j] = fmaf(__uint_as_float(r[b][j]), sc, acc[i < CPW ? i : 0][j]);
+                        }
                     }
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
-                buf ^= 1;
-                if (buf == 0) bphase ^= 1u;
+                if (++buf == S::NBUF) {
+                    buf = 0;
+                    bphase ^= 1u;
+                }
             }
             if (!ok) break;
 

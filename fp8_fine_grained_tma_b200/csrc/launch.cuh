@@ -34,6 +34,11 @@ int gemm_stage_bytes() {
         if (e != cudaSuccess) return e;                                                                        \
         const unsigned long long bit = 1ull << (dev & 63);                                                     \
         if (!(attr_set.load() & bit)) {                                                                        \
+            /* The in-kernel register split is only safe at exactly REGS_LAUNCH. */                            \
+            cudaFuncAttributes fa;                                                                             \
+            e = cudaFuncGetAttributes(&fa, fg8_gemm_kernel<BN>);                                               \
+            if (e != cudaSuccess) return e;                                                                    \
+            if (fa.numRegs != REGS_LAUNCH) return cudaErrorInvalidDeviceFunction;                              \
             e = cudaFuncSetAttribute(fg8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,         \
                                      kMaxDynamicSmem);                                                         \
             if (e != cudaSuccess) return e;                                                                    \

@@ -150,6 +150,14 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Empty asm that "rewrites" the registers: placed after tcgen05.wait::ld, it
+// keeps every use of a TMEM load's destination registers after the wait.
+__device__ __forceinline__ void reg_fence(uint32_t (&a)[16]) {
+    asm volatile(""
+                 : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
+                   "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]));
+}
+
 // tcgen05.wait::ld with the loaded registers tied through it, so no use of
 // them can be scheduled before the wait.
 __device__ __forceinline__ void tmem_wait_ld(uint32_t (&a)[16]) {
