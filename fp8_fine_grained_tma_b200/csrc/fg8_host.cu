@@ -18,7 +18,9 @@
 
 namespace fg8 {
 
-FG8_FOR_EACH_BN(FG8_DECLARE_LAUNCH)
+#define FG8_DECLARE_BOTH(BN) FG8_DECLARE_LAUNCH_ONE(BN, false) FG8_DECLARE_LAUNCH_ONE(BN, true)
+FG8_FOR_EACH_BN(FG8_DECLARE_BOTH)
+#undef FG8_DECLARE_BOTH
 
 // First error recorded by any GEMM kernel on this device: [0] = code,
 // [1] = (block << 8) | role.  Cleared by fg_get_last_device_status.
@@ -35,7 +37,6 @@ struct DeviceInfo {
     bool ready = false;
     int sm_count = 0;
     int cc_major = 0;
-    int regs_ok = -1;   // -1 unknown, 0 kernel build unusable, 1 ok
     int* status = nullptr;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -153,62 +154,99 @@ fg_status operand_map(const void* ptr, uint64_t K, uint64_t rows, uint64_t group
 }
 
 // ---- configuration -----------------------------------------------------------
-// Cost model for one candidate block width, in SM clock cycles:
-//   per K block a tile needs max(MMA, shared-memory read, L2->SM load) cycles;
-//   MMA = 2*BN (8192 E4M3 MAC/clk/SM), shared-memory reads of the MMA =
-//   (16 KiB of A + 128*BN of B) / 128 B/clk, loads = (valid A rows*128 +
-//   128*BN) / 64 B/clk.  Tiles per CTA = ceil(tiles / grid).  The whole job is
-//   also bounded below by its unique HBM bytes at ~3.5 KB/clk.
-double estimate_cycles(int rows_per_block_valid, long long tiles, int KB, int BN, int grid, double hbm_bytes) {
-    const double mma = 2.0 * BN;
-    const double smem = (16384.0 + 128.0 * BN) / 128.0;
-    const double load = (rows_per_block_valid * 128.0 + 128.0 * BN) / 64.0;
-    const double per_kb = std::max(mma, std::max(smem, load));
-    const double waves = static_cast<double>((tiles + grid - 1) / grid);
-    const double epilogue = 2.0 * BN + 600.0;
-    const double t_tiles = waves * (KB * per_kb + epilogue);
-    const double t_hbm = hbm_bytes / 3500.0;
-    return std::max(t_tiles, t_hbm) + 2000.0;
+// Cost model of one candidate (block width BN, 128-row tiles on one CTA or
+// 256-row tiles on a CTA pair), in SM clock cycles.  Per K block a tile needs
+//   max(MMA, promotion cycle, operand loads) cycles:
+//   MMA = 2*BN (8192 E4M3 MAC/clk/SM: each SM computes 128 x BN x 128),
+//   promotion cycle = 240 + 5*BN (measured on B200: the promotion warps' read /
+//           scale / accumulate / release cycle per K block, which the two to
+//           four TMEM accumulators cannot fully hide),
+//   loads = (A rows loaded * 128 + 128*BNL) / 44 B/clk (the L2 -> SM rate the
+//           kernel reaches when the tensor cores are idle),
+// with BNL = BN rows of B per CTA (BN/2 on a pair).  Tiles per CTA (pair) =
+// ceil(tiles / (SMs or SMs/2)); each tile adds an epilogue of ~2*BN + 800.
+// The job is bounded below by its unique HBM bytes at ~3.5 KB/clk.
+struct Choice {
+    int bn = 0;
+    bool pair = false;
+};
+
+double estimate_cycles(bool pair, int bn, long long row_tiles, int a_rows, int N, int K, int num_sms,
+                       double hbm_bytes) {
+    const int KB = K / BK;
+    const int bnl = pair ? bn / 2 : bn;
+    const long long tiles = row_tiles * ((N + bn - 1) / bn);
+    const int units = std::max(1, pair ? num_sms / 2 : num_sms);
+    const double waves = static_cast<double>((tiles + units - 1) / units);
+    const double mma = 2.0 * bn;
+    const double promotion = 240.0 + 5.0 * bn;
+    const double loads = (a_rows * 128.0 + 128.0 * bnl) / 44.0;
+    const double per_kb = std::max(mma, std::max(promotion, loads));
+    const double t_tiles = waves * (KB * per_kb + 2.0 * bn + 800.0);
+    return std::max(t_tiles, hbm_bytes / 3500.0) + 2000.0;
 }
 
-int choose_block_n(long long rows_total_blocks, int valid_rows_per_block, int N, int K, int num_sms,
-                   double hbm_bytes) {
+// rows: rows per row group; groups: row groups (masked: G, else 1); valid_rows:
+// expected rows that carry data per group (the masked hint, else rows).
+Choice choose_config(int layout, int rows, int groups, int valid_rows, int N, int K, int num_sms, double hbm_bytes) {
+    Choice best;
     const char* force = std::getenv("FG_FORCE_BLOCK_N");
-    if (force) {
-        int f = std::atoi(force);
-        if (f >= 16 && f <= 256 && f % 16 == 0) return f;
-    }
-    const int KB = K / BK;
-    int best = 16;
+    const char* force_pair = std::getenv("FG_FORCE_PAIR");
+    const int fbn = force ? std::atoi(force) : 0;
+    const int fpair = force_pair ? std::atoi(force_pair) : -1;
+    // CTA pairs halve each SM's B loads, but on B200 their cross-CTA handshake
+    // costs more than it saves for every workload measured so far, so they run
+    // only on request (FG_FORCE_PAIR=1).
+    const bool pair_ok = fpair == 1 && num_sms >= 2 && !(layout == LAYOUT_CONTIGUOUS && rows / BM > MAX_PAIR_LIST);
     double best_t = 1e300;
-    for (int bn = 16; bn <= 256; bn += 16) {
-        const long long tiles = rows_total_blocks * ((N + bn - 1) / bn);
-        const int grid = static_cast<int>(std::min<long long>(tiles, num_sms));
-        const double t = estimate_cycles(valid_rows_per_block, tiles, KB, bn, std::max(grid, 1), hbm_bytes);
-        if (t < best_t * 0.999 || (t <= best_t * 1.001 && bn > best)) {
-            if (t < best_t) best_t = t;
-            best = bn;
+    for (int pair = 0; pair <= 1; ++pair) {
+        if (pair && !pair_ok) continue;
+        if (fpair >= 0 && pair != fpair) continue;
+        for (int bn = pair ? 32 : 16; bn <= 256; bn += 16) {
+            if (fbn >= 16 && fbn <= 256 && fbn % 16 == 0 && bn != fbn) continue;
+            const int tile_m = pair ? 2 * BM : BM;
+            const long long row_tiles = static_cast<long long>(groups) * ((valid_rows + tile_m - 1) / tile_m);
+            const int a_rows = std::min(BM, std::max(1, valid_rows));
+            const double t = estimate_cycles(pair, bn, std::max(1ll, row_tiles), a_rows, N, K, num_sms, hbm_bytes);
+            if (t < best_t * 0.999 || (t <= best_t * 1.001 && (pair > (best.pair ? 1 : 0) || bn > best.bn))) {
+                if (t < best_t) best_t = t;
+                best.bn = bn;
+                best.pair = pair != 0;
+            }
         }
     }
     return best;
 }
 
-int stage_bytes_for(int bn) { return BM * BK + bn * BK; }
+int stage_bytes_for(int bn, bool pair) { return BM * BK + (pair ? bn / 2 : bn) * BK; }
 
-int choose_stages(int bn) {
-    const int sb = stage_bytes_for(bn);
+// At least MAX_NBUF stages: an MMA issuer then never waits on a stage barrier
+// more than one phase ahead (every block width fits 4 stages in 227 KiB).
+int choose_stages(int bn, bool pair) {
+    const int sb = stage_bytes_for(bn, pair);
     int s = 8;
-    while (s > 2 && gemm_smem_bytes(sb, s) > static_cast<size_t>(kMaxDynamicSmem)) --s;
+    while (s > MAX_NBUF && gemm_smem_bytes(sb, s) > static_cast<size_t>(kMaxDynamicSmem)) --s;
     return s;
 }
 
-fg_status launch_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
+template <int BN>
+cudaError_t launch_either(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
+                          size_t smem, cudaStream_t st) {
+    if constexpr (BN >= 32) {
+        if (pair) return launch_gemm<BN, true>(ta, tb, p, grid, smem, st);
+    } else {
+        if (pair) return cudaErrorInvalidValue;
+    }
+    return launch_gemm<BN, false>(ta, tb, p, grid, smem, st);
+}
+
+fg_status launch_bn(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
                     size_t smem, cudaStream_t st) {
     cudaError_t e = cudaErrorInvalidValue;
     switch (bn) {
 #define FG8_CASE(BNV) \
     case BNV:         \
-        e = launch_gemm<BNV>(ta, tb, p, grid, smem, st); \
+        e = launch_either<BNV>(pair, ta, tb, p, grid, smem, st); \
         break;
         FG8_FOR_EACH_BN(FG8_CASE)
 #undef FG8_CASE
@@ -238,19 +276,19 @@ fg_status run_gemm(int layout, const void* A, const float* sfa, const void* B, c
     const int KB = K / BK;
     const int NB = (N + 127) / 128;
     const int a_groups = layout == LAYOUT_MASKED ? G : 1;
-    const long long m_blocks = (rows + BM - 1) / BM;
-    const long long row_blocks_total = m_blocks * a_groups;
-    const int valid_rows = std::min(BM, std::max(1, valid_rows_hint));
-    const double hbm = static_cast<double>(a_groups) * rows * K + static_cast<double>(G) * N * K +
-                       2.0 * a_groups * rows * N;
-    const int bn = choose_block_n(row_blocks_total, valid_rows, N, K, num_sms, hbm);
-    const int stages = choose_stages(bn);
-    const size_t smem = gemm_smem_bytes(stage_bytes_for(bn), stages);
+    const double hbm = static_cast<double>(a_groups) * std::min(rows, std::max(1, valid_rows_hint)) * K +
+                       static_cast<double>(G) * N * K + 2.0 * a_groups * rows * N;
+    const Choice c = choose_config(layout, rows, a_groups, layout == LAYOUT_MASKED ? valid_rows_hint : rows, N, K,
+                                   num_sms, hbm);
+    const int bn = c.bn;
+    const int tile_m = c.pair ? 2 * BM : BM;
+    const int stages = choose_stages(bn, c.pair);
+    const size_t smem = gemm_smem_bytes(stage_bytes_for(bn, c.pair), stages);
 
     CUtensorMap ta, tb;
     st = operand_map(A, K, rows, a_groups, BM, &ta);
     if (st != FG_OK) return st;
-    st = operand_map(B, K, N, G, bn, &tb);
+    st = operand_map(B, K, N, G, c.pair ? bn / 2 : bn, &tb);
     if (st != FG_OK) return st;
 
     GemmParams p;
@@ -262,9 +300,9 @@ fg_status run_gemm(int layout, const void* A, const float* sfa, const void* B, c
     p.G = G;
     p.KB = KB;
     p.NB = NB;
-    p.num_m_blocks = static_cast<int>(m_blocks);
+    p.num_m_tiles = (rows + tile_m - 1) / tile_m;
     p.num_n_blocks = (N + bn - 1) / bn;
-    p.raster_m = 16;
+    p.raster_m = c.pair ? 8 : 16;
     p.stages = stages;
     p.sfa_ld = static_cast<int>(fg_get_tma_aligned_size(rows, 4));
     p.sfa = sfa;
@@ -275,9 +313,14 @@ fg_status run_gemm(int layout, const void* A, const float* sfa, const void* B, c
     p.status = dev->status;
     p.wait_limit_ns = g_wait_limit_ns.load();
 
-    long long tiles = row_blocks_total * p.num_n_blocks;
-    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(tiles, num_sms)));
-    return launch_bn(bn, ta, tb, p, grid, smem, stream);
+    // Upper bound of the tiles (the masked and contiguous schedulers may find fewer on the device).
+    const long long row_tiles = layout == LAYOUT_CONTIGUOUS ? (c.pair ? rows / BM : p.num_m_tiles)
+                                                            : static_cast<long long>(a_groups) * p.num_m_tiles;
+    const long long tiles = row_tiles * p.num_n_blocks;
+    const int units = c.pair ? num_sms / 2 : num_sms;
+    const long long used = std::max<long long>(1, std::min<long long>(tiles, units));
+    const int grid = static_cast<int>(c.pair ? 2 * used : used);
+    return launch_bn(bn, c.pair, ta, tb, p, grid, smem, stream);
 }
 
 __global__ void sfa_transform_kernel(const float* __restrict__ in, float* __restrict__ out, int G, int M, int KB,
@@ -454,7 +497,8 @@ int fg_query_block_n(int M, int N, int K) {
     if (current_device(&d) == FG_OK) sms = effective_sms(*d);
     else if (g_num_sms.load() > 0) sms = g_num_sms.load();
     const double hbm = static_cast<double>(M) * K + static_cast<double>(N) * K + 2.0 * M * N;
-    return choose_block_n((M + BM - 1) / BM, std::min(M, BM), N, K, sms, hbm);
+    const Choice c = choose_config(LAYOUT_NORMAL, M, 1, M, N, K, sms, hbm);
+    return c.pair ? -c.bn : c.bn;
 }
 
 }  // extern "C"

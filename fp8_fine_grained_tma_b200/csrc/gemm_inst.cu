@@ -1,5 +1,5 @@
-// gemm_inst.cu -- one instantiation of the GEMM kernel per build, selected by
-// -DFG8_BN=<block width>, so the sixteen block widths compile in parallel.
+// gemm_inst.cu -- the GEMM kernels of one block width, selected by
+// -DFG8_BN=<width>, so the sixteen block widths compile in parallel.
 #include "launch.cuh"
 
 #ifndef FG8_BN
@@ -7,5 +7,8 @@
 #endif
 
 namespace fg8 {
-FG8_DEFINE_LAUNCH(FG8_BN)
+FG8_DEFINE_LAUNCH_ONE(FG8_BN, false)
+#if FG8_BN >= 32
+FG8_DEFINE_LAUNCH_ONE(FG8_BN, true)
+#endif
 }  // namespace fg8

@@ -1,6 +1,6 @@
 // gemm_kernel.cuh -- persistent fine-grained-scaled FP8 GEMM for sm_100a.
 //
-// Computes, for each output tile of BM x BN,
+// Computes, for each output tile,
 //   D[m,n] = bf16( sum_kb (A_kb . B_kb^T)[m,n] * sfa[m,kb] * sfb[n/128,kb] )
 // which is the fine-grained ("DeepSeek-V3 style") scaling of the pages
 // (chujupifa.com "机器之心报道", opening summary; deepseek.csdn.net
@@ -9,18 +9,26 @@
 // tensor core, then scaled and added into FP32 on the CUDA cores;
 // chujupifa.com report, opening summary; ai.abqq.net, section 1 "架构优化").
 //
-// B200 design (not the pages' Hopper design):
-//   warp 8     TMA producer: one lane streams A [128 x 128] and B [BN x 128]
-//              E4M3 tiles into an S-stage shared-memory ring (128-byte swizzle).
-//   warp 9     MMA issuer: one lane issues 4 x tcgen05.mma kind::f8f6f4
-//              (M=128, N=BN, K=32) per K block into one of NBUF (2..4) TMEM
-//              accumulators, overwriting it at the block's first MMA.
+// B200 design (not the pages' Hopper design).  One CTA per SM, 12 warps:
+//   warp 8     TMA producer: one lane streams the CTA's A [128 x 128] and B
+//              [BNL x 128] E4M3 tiles into an S-stage shared-memory ring
+//              (128-byte swizzle).
+//   warps 9-10 MMA issuers: one lane each, taking turns by K block, issues
+//              4 x tcgen05.mma kind::f8f6f4 (K=32) per K block into one of NBUF
+//              (2..4) TMEM accumulators, overwriting it at the block's first MMA.
 //   warps 0-7  promotion + epilogue: two warpgroups split the tile's 16-column
 //              chunks; each thread owns one TMEM lane (= one output row), reads
 //              the block's partial sums with tcgen05.ld, multiplies by
-//              sfa[m,kb] * sfb[n/128,kb] and adds into FP32 registers, then
-//              after the last block converts to BF16 and stores the rows that
-//              may be written.
+//              sfa[m,kb] * sfb[n/128,kb] and adds into FP32 registers; after
+//              the last block it converts to BF16 and stores the rows that may
+//              be written.
+//   warp 11    idle (it completes the third warpgroup for the register split).
+// PAIR = false: the tile is 128 x BN and the CTA works alone (M=128 MMA).
+// PAIR = true:  two CTAs of a cluster share a 256 x BN tile (tcgen05
+//   cta_group::2, M=256): each loads its own 128 rows of A and its own half of
+//   the BN rows of B, the leader CTA issues the MMAs, and each CTA's TMEM holds
+//   its 128 rows x BN columns.  Each SM then moves 16 KiB + BN/2 * 128 bytes per
+//   K block instead of 16 KiB + BN * 128.  No load uses multicast.
 // Tiles are scheduled persistently (static stride over a raster-grouped tile
 // order); the contiguous and masked MoE layouts of the pages (game.3loumao.org
 // explainer, section "03 DeepSeek是如何创新的？") change only the tile -> (group,
@@ -38,7 +46,8 @@ constexpr int BM = 128;
 constexpr int BK = 128;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int PRODUCER_WARP = 8;
-constexpr int MMA_WARP = 9;
+constexpr int MMA_WARP = 9;                        // first MMA issuer (also allocates TMEM)
+constexpr int NUM_MMA_WARPS = 2;                   // warps MMA_WARP .. MMA_WARP + NUM_MMA_WARPS - 1 issue MMAs
 constexpr int NUM_THREADS = 384;                   // 3 warpgroups: 2 promotion, 1 producer/MMA
 // Register split (setmaxnreg, inside each role's own branch): every thread is
 // launched with REGS_LAUNCH registers; the producer warpgroup (warps 8..11)
@@ -54,6 +63,10 @@ constexpr int EPI_COLS = 32;                       // columns per staged piece
 constexpr int EPI_PITCH = EPI_COLS * 2 + 16;       // bytes per staged row (padding kills bank conflicts)
 constexpr int EPI_WARP_BYTES = 32 * EPI_PITCH;     // staging bytes per epilogue warp
 constexpr int A_TILE_BYTES = BM * BK;              // 16 KiB
+// Contiguous layout, CTA pairs: the 128-row blocks that start a pair tile are
+// listed in shared memory (one 16-bit block index each).
+constexpr int MAX_PAIR_LIST = 4096;
+constexpr int PAIR_LIST_BYTES = MAX_PAIR_LIST * 2;
 
 enum : int { LAYOUT_NORMAL = 0, LAYOUT_CONTIGUOUS = 1, LAYOUT_MASKED = 2 };
 
@@ -65,9 +78,9 @@ struct GemmParams {
     int rows;          // rows per group: M (normal), M_tot (contiguous), M_max (masked)
     int N, K, G;
     int KB, NB;        // K / 128, ceil(N / 128)
-    int num_m_blocks;  // ceil(rows / BM)
+    int num_m_tiles;   // row tiles per group: ceil(rows / (128 or 256))
     int num_n_blocks;  // ceil(N / BN)
-    int raster_m;      // row blocks per raster group
+    int raster_m;      // row tiles per raster group
     int stages;
     int sfa_ld;        // M_pad: stride (floats) between K blocks of the MN-major sfa
     const float* sfa;  // [G or 1][KB][sfa_ld]
@@ -81,12 +94,15 @@ struct GemmParams {
 
 __host__ __device__ constexpr int ceil_div_c(int a, int b) { return (a + b - 1) / b; }
 
-template <int BN>
+template <int BN, bool PAIR>
 struct GemmShape {
     static constexpr int NC = BN / 16;                  // 16-column chunks in a tile
     static constexpr int CPW = (NC + 1) / 2;            // chunks per promotion warpgroup
-    static constexpr int B_TILE_BYTES = BN * BK;
+    static constexpr int BNL = PAIR ? BN / 2 : BN;      // B rows this CTA loads per K block
+    static constexpr int TILE_M = PAIR ? 2 * BM : BM;   // rows of a tile
+    static constexpr int B_TILE_BYTES = BNL * BK;
     static constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
+    static constexpr int TX_BYTES = PAIR ? 2 * STAGE_BYTES : STAGE_BYTES;   // expected on the (leader's) full barrier
     static constexpr int ACC_STRIDE = (BN + 31) / 32 * 32;   // TMEM columns per accumulator
     // As many K-block accumulators as TMEM holds (at most 4): the MMA issuer may
     // run NBUF - 1 blocks ahead of the promotion warps.
@@ -97,33 +113,48 @@ struct GemmShape {
                                      : TMEM_USED <= 128 ? 128
                                      : TMEM_USED <= 256 ? 256
                                                         : 512;
-    static_assert(NBUF >= 2, "need two accumulators");
+    static constexpr int TEMPTY_COUNT = PAIR ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN must be a multiple of 16 in [16, 256]");
+    static_assert(!PAIR || BN >= 32, "a CTA pair needs at least 16 B rows per CTA");
+    static_assert(NBUF >= 2, "need two accumulators");
+    // An issuer waits on an accumulator / stage barrier for the phase right
+    // after the one its previous K block used; with more issuers than
+    // accumulators it could wait two phases ahead and see a stale completion.
+    // (The host also keeps the stage count >= NBUF for the same reason.)
+    static_assert(NUM_MMA_WARPS <= NBUF, "more MMA issuers than TMEM accumulators");
 };
 
 // Dynamic shared memory layout (after aligning the base to 1024 bytes):
-//   [stages x (A tile | B tile)] [8 x epilogue staging] [barriers] [tmem slot, abort flag]
+//   [stages x (A tile | B tile)] [8 x epilogue staging] [pair list] [barriers] [tmem slot, abort flag, list count]
 constexpr int MAX_NBUF = 4;
 __host__ __device__ constexpr size_t gemm_smem_bytes(int stage_bytes, int stages) {
-    return 1024 + static_cast<size_t>(stages) * stage_bytes + NUM_EPI_WARPS * EPI_WARP_BYTES +
+    return 1024 + static_cast<size_t>(stages) * stage_bytes + NUM_EPI_WARPS * EPI_WARP_BYTES + PAIR_LIST_BYTES +
            (2 * stages + 2 * MAX_NBUF + 1) * 8 + 16;
 }
 
 struct TileInfo {
     int g;       // group of B / sfb (expert); for the masked layout also of A / D
-    int m_blk;
+    int row0;    // first row (within the group) of this CTA's 128-row slice of the tile
     int n_blk;
 };
 
-// Enumerates the tiles of this CTA.  Every role builds its own copy and walks
-// the same sequence, so no role has to tell another which tile comes next.
+// Enumerates the tiles of this CTA (or CTA pair).  Every role builds its own
+// copy and walks the same sequence, so no role tells another which tile is next.
+template <bool PAIR>
 struct TileScheduler {
     int next;
-    int mg, mbase, mtiles, mblocks;   // masked layout cursor
+    int stride;
+    int rank;                          // CTA rank within the pair (0 when alone)
+    int mg, mbase, mtiles, mtiles_m;   // masked layout cursor
+    const uint16_t* pair_list;         // contiguous layout with pairs
+    int pair_count;
 
-    __device__ explicit TileScheduler() : next(blockIdx.x), mg(0), mbase(0), mtiles(-1), mblocks(0) {}
+    __device__ TileScheduler(int unit, int num_units, int rank_, const uint16_t* list, int count)
+        : next(unit), stride(num_units), rank(rank_), mg(0), mbase(0), mtiles(-1), mtiles_m(0), pair_list(list),
+          pair_count(count) {}
 
     __device__ bool get(const GemmParams& p, TileInfo& t) {
+        constexpr int TILE_M = PAIR ? 2 * BM : BM;
         if (p.layout == LAYOUT_MASKED) {
             const int idx = next;
             while (true) {
@@ -131,8 +162,8 @@ struct TileScheduler {
                 if (mtiles < 0) {
                     int mm = __ldg(p.masked_m + mg);
                     mm = mm < 0 ? 0 : (mm > p.rows ? p.rows : mm);
-                    mblocks = ceil_div_c(mm, BM);
-                    mtiles = mblocks * p.num_n_blocks;
+                    mtiles_m = ceil_div_c(mm, TILE_M);
+                    mtiles = mtiles_m * p.num_n_blocks;
                 }
                 if (idx < mbase + mtiles) break;
                 mbase += mtiles;
@@ -141,25 +172,42 @@ struct TileScheduler {
             }
             const int local = idx - mbase;
             t.g = mg;
-            t.m_blk = local % mblocks;   // row blocks of one column block run side by side
-            t.n_blk = local / mblocks;
-            next += gridDim.x;
+            t.row0 = (local % mtiles_m) * TILE_M + rank * BM;   // row tiles of one column block run side by side
+            t.n_blk = local / mtiles_m;
+            next += stride;
             return true;
         }
-        const int total = p.num_m_blocks * p.num_n_blocks;
-        while (next < total) {
+        if (PAIR && p.layout == LAYOUT_CONTIGUOUS) {
+            const int total = pair_count * p.num_n_blocks;
+            if (next >= total) return false;
             const int idx = next;
-            next += gridDim.x;
+            next += stride;
             const int per_group = p.raster_m * p.num_n_blocks;
             const int grp = idx / per_group;
             const int first_m = grp * p.raster_m;
-            const int gm = min(p.raster_m, p.num_m_blocks - first_m);
+            const int gm = min(p.raster_m, pair_count - first_m);
             const int local = idx - grp * per_group;
-            t.m_blk = first_m + local % gm;
+            const int blk = pair_list[first_m + local % gm];
             t.n_blk = local / gm;
+            t.row0 = (blk + rank) * BM;
+            t.g = __ldg(p.m_indices + blk * BM);
+            return true;
+        }
+        const int total = p.num_m_tiles * p.num_n_blocks;
+        while (next < total) {
+            const int idx = next;
+            next += stride;
+            const int per_group = p.raster_m * p.num_n_blocks;
+            const int grp = idx / per_group;
+            const int first_m = grp * p.raster_m;
+            const int gm = min(p.raster_m, p.num_m_tiles - first_m);
+            const int local = idx - grp * per_group;
+            const int m_tile = first_m + local % gm;
+            t.n_blk = local / gm;
+            t.row0 = m_tile * TILE_M + rank * BM;
             t.g = 0;
             if (p.layout == LAYOUT_CONTIGUOUS) {
-                const int e = __ldg(p.m_indices + t.m_blk * BM);
+                const int e = __ldg(p.m_indices + m_tile * BM);
                 if (e < 0 || e >= p.G) continue;   // a block of padding rows only: nothing to do
                 t.g = e;
             }
@@ -170,11 +218,17 @@ struct TileScheduler {
 };
 
 // Wait result: 0 = completed, 1 = another role aborted, 2 = this wait timed out.
+// The thread is parked by the hardware (mbarrier suspend hint, at most 1 ms per
+// try) rather than spinning, so waiting roles take no issue slots or shared
+// memory bandwidth from the MMA; the abort flag and the time limit are checked
+// each time a try expires.
 __device__ __forceinline__ int wait_bar(uint64_t* bar, uint32_t parity, uint64_t limit_ns, volatile int* abort_flag) {
-    if (ptx::mbar_try_wait(bar, parity)) return 0;
+    if (ptx::mbar_test_wait(bar, parity)) return 0;   // fast path: the phase is already complete
+    const uint32_t hint = limit_ns < 1000000ull ? static_cast<uint32_t>(limit_ns) : 1000000u;
+    if (ptx::mbar_try_wait_suspend(bar, parity, hint)) return 0;
     const uint64_t t0 = ptx::globaltimer();
     while (true) {
-        if (ptx::mbar_try_wait(bar, parity)) return 0;
+        if (ptx::mbar_try_wait_suspend(bar, parity, hint)) return 0;
         if (*abort_flag) return 1;
         if (ptx::globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
@@ -192,32 +246,69 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int BN>
+// Contiguous layout with CTA pairs: list, in row order, the 128-row blocks that
+// start a pair tile.  A pair starts at every even offset of a run of blocks
+// carrying the same expert tag (tag of a block = tag of its first row); the
+// second block of a pair may belong to another expert or be padding, and then
+// that CTA's rows are simply not stored.  Run by warp 0; `tags` is scratch
+// shared memory for one int per block.  Returns the number of pairs.
+__device__ __forceinline__ int build_pair_list(const GemmParams& p, int* tags, uint16_t* list) {
+    const int lane = threadIdx.x % 32;
+    const int nblk = p.rows / BM;
+    for (int b = lane; b < nblk; b += 32) {
+        const int e = __ldg(p.m_indices + b * BM);
+        tags[b] = (e < 0 || e >= p.G) ? -1 : e;
+    }
+    __syncwarp();
+    int count = 0;
+    for (int base = 0; base < nblk; base += 32) {
+        const int b = base + lane;
+        bool start = false;
+        if (b < nblk && tags[b] >= 0) {
+            int run = 0;   // blocks of the same tag directly before b
+            while (b - run - 1 >= 0 && tags[b - run - 1] == tags[b]) ++run;
+            start = (run % 2) == 0;
+        }
+        const uint32_t mask = __ballot_sync(0xffffffffu, start);
+        const int pos = count + __popc(mask & ((1u << lane) - 1u));
+        if (start && pos < MAX_PAIR_LIST) list[pos] = static_cast<uint16_t>(b);
+        count += __popc(mask);
+    }
+    return count < MAX_PAIR_LIST ? count : MAX_PAIR_LIST;
+}
+
+template <int BN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fg8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const GemmParams p) {
-    using S = GemmShape<BN>;
+    using S = GemmShape<BN, PAIR>;
     constexpr int NC = S::NC;
     constexpr int CPW = S::CPW;
     constexpr int LB = CPW <= 4 ? CPW : 4;   // chunks read from TMEM per wait
-    constexpr uint32_t IDESC = ptx::idesc_e4m3_f32(BM, BN);
+    constexpr uint32_t IDESC = ptx::idesc_e4m3_f32(S::TILE_M, BN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stage_base = smem;
     uint8_t* epi_base = smem + static_cast<size_t>(p.stages) * S::STAGE_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(epi_base + NUM_EPI_WARPS * EPI_WARP_BYTES);
+    uint16_t* pair_list = reinterpret_cast<uint16_t*>(epi_base + NUM_EPI_WARPS * EPI_WARP_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(pair_list) + PAIR_LIST_BYTES);
     uint64_t* empty = full + p.stages;
     uint64_t* tfull = empty + p.stages;
     uint64_t* tempty = tfull + S::NBUF;
     uint64_t* done_bar = tempty + S::NBUF;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* pair_count_slot = reinterpret_cast<int*>(tmem_slot + 2);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const uint64_t limit = p.wait_limit_ns;
     const uint64_t drain_limit = 2000000000ull;   // 2 s: copies in flight always finish
+    const int rank = PAIR ? static_cast<int>(ptx::cluster_ctarank()) : 0;
+    const bool leader = rank == 0;
+    const int unit = PAIR ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+    const int num_units = PAIR ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
 
     if (warp == PRODUCER_WARP && lane == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -226,44 +317,63 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int b = 0; b < S::NBUF; ++b) {
             ptx::mbar_init(&tfull[b], 1);
-            ptx::mbar_init(&tempty[b], NUM_EPI_WARPS);
+            ptx::mbar_init(&tempty[b], S::TEMPTY_COUNT);
         }
-        ptx::mbar_init(done_bar, 1);
+        ptx::mbar_init(done_bar, NUM_MMA_WARPS);
         *abort_flag = 0;
         ptx::fence_mbarrier_init();
         ptx::prefetch_tensormap(&tmA);
         ptx::prefetch_tensormap(&tmB);
     }
     if (warp == MMA_WARP) {
-        ptx::tmem_alloc(tmem_slot, S::TMEM_COLS);
-        ptx::tmem_relinquish();
+        if constexpr (PAIR) {
+            ptx::tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
+            ptx::tmem_relinquish_pair();
+        } else {
+            ptx::tmem_alloc(tmem_slot, S::TMEM_COLS);
+            ptx::tmem_relinquish();
+        }
+    }
+    if (PAIR && p.layout == LAYOUT_CONTIGUOUS && warp == 0) {
+        // The stage ring is free until the roles start: use it for the tags.
+        const int n = build_pair_list(p, reinterpret_cast<int*>(stage_base), pair_list);
+        if (lane == 0) *pair_count_slot = n;
     }
     ptx::tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) ptx::cluster_sync();   // peer barriers initialised, TMEM of both CTAs allocated
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const int pair_count = (PAIR && p.layout == LAYOUT_CONTIGUOUS) ? *pair_count_slot : 0;
 
     if (warp >= NUM_EPI_WARPS) {
       ptx::setmaxnreg_dec<REGS_PRODUCER>();
       if (warp == PRODUCER_WARP) {
         if (lane == 0) {
-            TileScheduler sch;
+            TileScheduler<PAIR> sch(unit, num_units, rank, pair_list, pair_count);
             TileInfo t;
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;           // loads issued so far (for the drain below)
             int w = 0;
             while (w == 0 && sch.get(p, t)) {
-                const int a_row = t.m_blk * BM;
                 const int a_g = p.layout == LAYOUT_MASKED ? t.g : 0;
-                const int b_row = t.n_blk * BN;
+                const int b_row = t.n_blk * BN + rank * S::BNL;
                 for (int kb = 0; kb < p.KB; ++kb) {
                     w = wait_bar(&empty[stage], phase ^ 1u, limit, abort_flag);
                     if (w) break;
                     uint8_t* sa = stage_base + static_cast<size_t>(stage) * S::STAGE_BYTES;
-                    ptx::mbar_arrive_expect_tx(&full[stage], S::STAGE_BYTES);
-                    ptx::tma_load_3d(sa, &tmA, &full[stage], kb * BK, a_row, a_g);
-                    ptx::tma_load_3d(sa + A_TILE_BYTES, &tmB, &full[stage], kb * BK, b_row, t.g);
+                    if constexpr (PAIR) {
+                        // Both CTAs' loads complete on the leader's full barrier.
+                        const uint32_t bar = ptx::mapa_shared(ptx::smem_addr(&full[stage]), 0);
+                        if (leader) ptx::mbar_arrive_expect_tx(&full[stage], S::TX_BYTES);
+                        ptx::tma_load_3d_pair(sa, &tmA, bar, kb * BK, t.row0, a_g);
+                        ptx::tma_load_3d_pair(sa + A_TILE_BYTES, &tmB, bar, kb * BK, b_row, t.g);
+                    } else {
+                        ptx::mbar_arrive_expect_tx(&full[stage], S::TX_BYTES);
+                        ptx::tma_load_3d(sa, &tmA, &full[stage], kb * BK, t.row0, a_g);
+                        ptx::tma_load_3d(sa + A_TILE_BYTES, &tmB, &full[stage], kb * BK, b_row, t.g);
+                    }
                     ++issued;
                     if (++stage == p.stages) {
                         stage = 0;
@@ -272,54 +382,73 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             }
             if (w == 2) record_error(p.status, ERR_TIMEOUT, ROLE_PRODUCER);
-            // Let every copy still in flight land before the CTA can exit.
-            // The last p.stages loads went to stages stage, stage+1, ... (mod p.stages)
-            // with the parity of the fill they belong to.
-            {
+            if (!PAIR || leader) {
+                // Let every copy still in flight land before the CTA can exit:
+                // walk back over the last p.stages loads (stage, parity).
                 int s = stage;
                 uint32_t ph = phase;
-                for (int i = 0; i < p.stages; ++i) {
-                    // walk back: (s, ph) after the loop are those of the oldest of the last loads
+                for (int i = 0; i < p.stages && issued - 1 - i >= 0; ++i) {
                     if (s == 0) {
                         s = p.stages - 1;
                         ph ^= 1u;
                     } else {
                         --s;
                     }
-                    if (issued - 1 - i < 0) break;
                     ptx::mbar_wait(&full[s], ph, drain_limit);
                 }
+            } else if (w != 0) {
+                // The peer's loads complete on the leader's barriers, which it
+                // cannot wait on: after an abort give them time to land.
+                for (int i = 0; i < 200; ++i) __nanosleep(1000);
             }
         }
-      } else if (warp == MMA_WARP) {
-        if (lane == 0) {
-            TileScheduler sch;
+      } else if (warp < MMA_WARP + NUM_MMA_WARPS) {
+        // K blocks are independent (each accumulates into its own TMEM buffer),
+        // so NUM_MMA_WARPS issuers take turns: issuer j handles the global
+        // K-block sequence numbers g with g % NUM_MMA_WARPS == j.  This hides
+        // the long per-thread latency of the barrier waits, the fence and each
+        // tcgen05 issue behind another issuer's work.
+        const int j = warp - MMA_WARP;
+        if (lane == 0 && (!PAIR || leader)) {
+            TileScheduler<PAIR> sch(unit, num_units, rank, pair_list, pair_count);
             TileInfo t;
             int stage = 0;
             uint32_t phase = 0;
             int buf = 0;
             uint32_t bphase = 0;
             int w = 0;
+            int g = 0;
             while (w == 0 && sch.get(p, t)) {
-                for (int kb = 0; kb < p.KB; ++kb) {
-                    w = wait_bar(&tempty[buf], bphase ^ 1u, limit, abort_flag);
-                    if (w) break;
-                    ptx::tc_fence_after();
-                    w = wait_bar(&full[stage], phase, limit, abort_flag);
-                    if (w) break;
-                    ptx::tc_fence_after();
-                    const uint32_t a_addr = ptx::smem_addr(stage_base + static_cast<size_t>(stage) * S::STAGE_BYTES);
-                    const uint64_t adesc = ptx::smem_desc_sw128(a_addr);
-                    const uint64_t bdesc = ptx::smem_desc_sw128(a_addr + A_TILE_BYTES);
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * S::ACC_STRIDE);
+                for (int kb = 0; kb < p.KB; ++kb, ++g) {
+                    if (g % NUM_MMA_WARPS == j) {
+                        w = wait_bar(&tempty[buf], bphase ^ 1u, limit, abort_flag);
+                        if (w) break;
+                        w = wait_bar(&full[stage], phase, limit, abort_flag);
+                        if (w) break;
+                        ptx::tc_fence_after();
+                        const uint32_t a_addr =
+                            ptx::smem_addr(stage_base + static_cast<size_t>(stage) * S::STAGE_BYTES);
+                        const uint64_t adesc = ptx::smem_desc_sw128(a_addr);
+                        const uint64_t bdesc = ptx::smem_desc_sw128(a_addr + A_TILE_BYTES);
+                        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * S::ACC_STRIDE);
 #pragma unroll
-                    for (int j = 0; j < BK / 32; ++j) {
-                        // K step j: 32 E4M3 = 32 bytes further along the swizzled 128-byte row.
-                        ptx::mma_f8f6f4(d_tmem, adesc + static_cast<uint64_t>(j * 2), bdesc + static_cast<uint64_t>(j * 2),
-                                        IDESC, j > 0 ? 1u : 0u);
+                        for (int k = 0; k < BK / 32; ++k) {
+                            // K step k: 32 E4M3 = 32 bytes further along the swizzled 128-byte row.
+                            if constexpr (PAIR)
+                                ptx::mma_f8f6f4_pair(d_tmem, adesc + static_cast<uint64_t>(k * 2),
+                                                     bdesc + static_cast<uint64_t>(k * 2), IDESC, k > 0 ? 1u : 0u);
+                            else
+                                ptx::mma_f8f6f4(d_tmem, adesc + static_cast<uint64_t>(k * 2),
+                                                bdesc + static_cast<uint64_t>(k * 2), IDESC, k > 0 ? 1u : 0u);
+                        }
+                        if constexpr (PAIR) {
+                            ptx::mma_commit_pair(&empty[stage], 0x3);
+                            ptx::mma_commit_pair(&tfull[buf], 0x3);
+                        } else {
+                            ptx::mma_commit(&empty[stage]);
+                            ptx::mma_commit(&tfull[buf]);
+                        }
                     }
-                    ptx::mma_commit(&empty[stage]);
-                    ptx::mma_commit(&tfull[buf]);
                     if (++stage == p.stages) {
                         stage = 0;
                         phase ^= 1u;
@@ -331,8 +460,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             }
             if (w == 2) record_error(p.status, ERR_TIMEOUT, ROLE_MMA);
-            // Every MMA issued above must finish before TMEM is released.
-            ptx::mma_commit(done_bar);
+            // Every MMA issued above must finish before TMEM is released
+            // (done_bar completes once every issuer's commit has arrived).
+            if constexpr (PAIR) ptx::mma_commit_pair(done_bar, 0x1);
+            else ptx::mma_commit(done_bar);
             ptx::mbar_wait(done_bar, 0, drain_limit);
         }
       }
@@ -346,13 +477,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int chunk0 = wg * CPW;                  // first 16-column chunk of this warpgroup
         uint8_t* stg = epi_base + warp * EPI_WARP_BYTES;
 
-        TileScheduler sch;
+        TileScheduler<PAIR> sch(unit, num_units, rank, pair_list, pair_count);
         TileInfo t;
         int buf = 0;
         uint32_t bphase = 0;
         bool ok = true;
         while (ok && sch.get(p, t)) {
-            const int row = t.m_blk * BM + row_in_tile;
+            const int row = t.row0 + row_in_tile;
             const bool row_in = row < p.rows;
             const int a_g = p.layout == LAYOUT_MASKED ? t.g : 0;
             const float* sfa_p = p.sfa + static_cast<size_t>(a_g) * p.KB * p.sfa_ld + row;
@@ -363,24 +494,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int nb_hi = min(nb_lo + 1, p.NB - 1);
             const int split_col = (my_n0 / 128 + 1) * 128;   // chunk columns at or past this use nb_hi
 
-            float acc[CPW][16];
+            // Column pairs: the promotion uses the packed FP32 FMA (two FMAs per
+            // instruction, each rounded to nearest as a scalar fmaf would be).
+            float2 acc[CPW][8];
 #pragma unroll
             for (int i = 0; i < CPW; ++i)
 #pragma unroll
-                for (int j = 0; j < 16; ++j) acc[i][j] = 0.0f;
+                for (int j = 0; j < 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
 
-            float sa_n = row_in ? __ldg(sfa_p) : 0.0f;
-            float sl_n = __ldg(sfb_p + static_cast<size_t>(nb_lo) * p.KB);
-            float sh_n = __ldg(sfb_p + static_cast<size_t>(nb_hi) * p.KB);
+            // Scales are fetched SCALE_AHEAD K blocks ahead into a small register
+            // ring, so a block's scale products never wait on a global load.
+            constexpr int SCALE_AHEAD = 3;
+            const float* sfb_lo = sfb_p + static_cast<size_t>(nb_lo) * p.KB;
+            const float* sfb_hi = sfb_p + static_cast<size_t>(nb_hi) * p.KB;
+            float ra[SCALE_AHEAD], rl[SCALE_AHEAD], rh[SCALE_AHEAD];
+#pragma unroll
+            for (int q = 0; q < SCALE_AHEAD; ++q) {
+                const int kq = q < p.KB ? q : p.KB - 1;
+                ra[q] = row_in ? __ldg(sfa_p + static_cast<size_t>(kq) * p.sfa_ld) : 0.0f;
+                rl[q] = __ldg(sfb_lo + kq);
+                rh[q] = __ldg(sfb_hi + kq);
+            }
             for (int kb = 0; kb < p.KB; ++kb) {
-                const float sa = sa_n, sl = sl_n, sh = sh_n;
-                if (kb + 1 < p.KB) {   // prefetch the next block's scales
-                    sa_n = row_in ? __ldg(sfa_p + static_cast<size_t>(kb + 1) * p.sfa_ld) : 0.0f;
-                    sl_n = __ldg(sfb_p + static_cast<size_t>(nb_lo) * p.KB + kb + 1);
-                    sh_n = __ldg(sfb_p + static_cast<size_t>(nb_hi) * p.KB + kb + 1);
+                const float s_lo = ra[0] * rl[0];
+                const float s_hi = ra[0] * rh[0];
+#pragma unroll
+                for (int q = 0; q + 1 < SCALE_AHEAD; ++q) {
+                    ra[q] = ra[q + 1];
+                    rl[q] = rl[q + 1];
+                    rh[q] = rh[q + 1];
                 }
-                const float s_lo = sa * sl;
-                const float s_hi = sa * sh;
+                {
+                    const int kq = kb + SCALE_AHEAD < p.KB ? kb + SCALE_AHEAD : p.KB - 1;
+                    ra[SCALE_AHEAD - 1] = row_in ? __ldg(sfa_p + static_cast<size_t>(kq) * p.sfa_ld) : 0.0f;
+                    rl[SCALE_AHEAD - 1] = __ldg(sfb_lo + kq);
+                    rh[SCALE_AHEAD - 1] = __ldg(sfb_hi + kq);
+                }
                 int w = 0;
                 if (lane == 0) w = wait_bar(&tfull[buf], bphase, limit, abort_flag);
                 w = __shfl_sync(0xffffffffu, w, 0);
@@ -410,15 +559,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const int c = chunk0 + i;
                         if (i < CPW && c < NC) {
                             const float sc = (n0 + c * 16 >= split_col) ? s_hi : s_lo;
+                            const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                acc[i < CPW ? i : 0][j] = fmaf(__uint_as_float(r[b][j]), sc, acc[i < CPW ? i : 0][j]);
+                            for (int j = 0; j < 8; ++j) {
+                                const float2 v = make_float2(__uint_as_float(r[b][2 * j]), __uint_as_float(r[b][2 * j + 1]));
+                                acc[i < CPW ? i : 0][j] = __ffma2_rn(v, sc2, acc[i < CPW ? i : 0][j]);
+                            }
                         }
                     }
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+                if (lane == 0) {
+                    if constexpr (PAIR) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_addr(&tempty[buf]), 0));
+                    else ptx::mbar_arrive(&tempty[buf]);
+                }
                 if (++buf == S::NBUF) {
                     buf = 0;
                     bphase ^= 1u;
@@ -439,53 +594,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             const uint32_t rows_mask = __ballot_sync(0xffffffffu, row_ok);
             __nv_bfloat16* Dg = p.D + (p.layout == LAYOUT_MASKED ? static_cast<size_t>(t.g) * p.rows * p.N : 0);
-            const int warp_row0 = t.m_blk * BM + quarter * 32;
+            const int warp_row0 = t.row0 + quarter * 32;
+            if (rows_mask != 0u) {
 #pragma unroll
-            for (int i = 0; i < CPW; i += 2) {
-                const int c0 = chunk0 + i;
-                if (c0 >= NC) break;
-                const bool has1 = (i + 1 < CPW) && (c0 + 1 < NC);
-                uint8_t* myrow = stg + lane * EPI_PITCH;
-                {
-                    uint4 v0, v1;
-                    v0.x = pack_bf16x2(acc[i][0], acc[i][1]);
-                    v0.y = pack_bf16x2(acc[i][2], acc[i][3]);
-                    v0.z = pack_bf16x2(acc[i][4], acc[i][5]);
-                    v0.w = pack_bf16x2(acc[i][6], acc[i][7]);
-                    v1.x = pack_bf16x2(acc[i][8], acc[i][9]);
-                    v1.y = pack_bf16x2(acc[i][10], acc[i][11]);
-                    v1.z = pack_bf16x2(acc[i][12], acc[i][13]);
-                    v1.w = pack_bf16x2(acc[i][14], acc[i][15]);
-                    *reinterpret_cast<uint4*>(myrow) = v0;
-                    *reinterpret_cast<uint4*>(myrow + 16) = v1;
-                }
-                if (has1) {
-                    const int i1 = (i + 1) < CPW ? i + 1 : i;
-                    uint4 v0, v1;
-                    v0.x = pack_bf16x2(acc[i1][0], acc[i1][1]);
-                    v0.y = pack_bf16x2(acc[i1][2], acc[i1][3]);
-                    v0.z = pack_bf16x2(acc[i1][4], acc[i1][5]);
-                    v0.w = pack_bf16x2(acc[i1][6], acc[i1][7]);
-                    v1.x = pack_bf16x2(acc[i1][8], acc[i1][9]);
-                    v1.y = pack_bf16x2(acc[i1][10], acc[i1][11]);
-                    v1.z = pack_bf16x2(acc[i1][12], acc[i1][13]);
-                    v1.w = pack_bf16x2(acc[i1][14], acc[i1][15]);
-                    *reinterpret_cast<uint4*>(myrow + 32) = v0;
-                    *reinterpret_cast<uint4*>(myrow + 48) = v1;
-                }
-                __syncwarp();
-                const int units = has1 ? 4 : 2;     // 16-byte units per staged row
-                const int col_base = n0 + c0 * 16;
-                for (int q = lane; q < 32 * units; q += 32) {
-                    const int r = q / units;
-                    const int u = q - r * units;
-                    const int gcol = col_base + u * 8;
-                    if (((rows_mask >> r) & 1u) && gcol < p.N) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(stg + r * EPI_PITCH + u * 16);
-                        *reinterpret_cast<uint4*>(Dg + static_cast<size_t>(warp_row0 + r) * p.N + gcol) = v;
+                for (int i = 0; i < CPW; i += 2) {
+                    const int c0 = chunk0 + i;
+                    if (c0 >= NC) break;
+                    const bool has1 = (i + 1 < CPW) && (c0 + 1 < NC);
+                    uint8_t* myrow = stg + lane * EPI_PITCH;
+                    {
+                        uint4 v0, v1;
+                        v0.x = pack_bf16x2(acc[i][0].x, acc[i][0].y);
+                        v0.y = pack_bf16x2(acc[i][1].x, acc[i][1].y);
+                        v0.z = pack_bf16x2(acc[i][2].x, acc[i][2].y);
+                        v0.w = pack_bf16x2(acc[i][3].x, acc[i][3].y);
+                        v1.x = pack_bf16x2(acc[i][4].x, acc[i][4].y);
+                        v1.y = pack_bf16x2(acc[i][5].x, acc[i][5].y);
+                        v1.z = pack_bf16x2(acc[i][6].x, acc[i][6].y);
+                        v1.w = pack_bf16x2(acc[i][7].x, acc[i][7].y);
+                        *reinterpret_cast<uint4*>(myrow) = v0;
+                        *reinterpret_cast<uint4*>(myrow + 16) = v1;
                     }
+                    if (has1) {
+                        const int i1 = (i + 1) < CPW ? i + 1 : i;
+                        uint4 v0, v1;
+                        v0.x = pack_bf16x2(acc[i1][0].x, acc[i1][0].y);
+                        v0.y = pack_bf16x2(acc[i1][1].x, acc[i1][1].y);
+                        v0.z = pack_bf16x2(acc[i1][2].x, acc[i1][2].y);
+                        v0.w = pack_bf16x2(acc[i1][3].x, acc[i1][3].y);
+                        v1.x = pack_bf16x2(acc[i1][4].x, acc[i1][4].y);
+                        v1.y = pack_bf16x2(acc[i1][5].x, acc[i1][5].y);
+                        v1.z = pack_bf16x2(acc[i1][6].x, acc[i1][6].y);
+                        v1.w = pack_bf16x2(acc[i1][7].x, acc[i1][7].y);
+                        *reinterpret_cast<uint4*>(myrow + 32) = v0;
+                        *reinterpret_cast<uint4*>(myrow + 48) = v1;
+                    }
+                    __syncwarp();
+                    const int units = has1 ? 4 : 2;     // 16-byte units per staged row
+                    const int col_base = n0 + c0 * 16;
+                    for (int q = lane; q < 32 * units; q += 32) {
+                        const int r = q / units;
+                        const int u = q - r * units;
+                        const int gcol = col_base + u * 8;
+                        if (((rows_mask >> r) & 1u) && gcol < p.N) {
+                            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * EPI_PITCH + u * 16);
+                            *reinterpret_cast<uint4*>(Dg + static_cast<size_t>(warp_row0 + r) * p.N + gcol) = v;
+                        }
+                    }
+                    __syncwarp();
                 }
-                __syncwarp();
             }
         }
     }
@@ -493,9 +650,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
     ptx::tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) ptx::cluster_sync();   // the leader's MMAs read the peer's shared memory until here
     if (warp == MMA_WARP) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem_base, S::TMEM_COLS);
+        if constexpr (PAIR) ptx::tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
+        else ptx::tmem_dealloc(tmem_base, S::TMEM_COLS);
     }
 }
 

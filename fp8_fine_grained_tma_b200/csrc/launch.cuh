@@ -1,4 +1,4 @@
-// launch.cuh -- the launcher each kernel instantiation exports to the host code.
+// launch.cuh -- the launchers each kernel instantiation exports to the host code.
 #pragma once
 
 #include <cuda.h>
@@ -13,46 +13,77 @@ namespace fg8 {
 // Largest dynamic shared memory a CTA may request on sm_100 (227 KiB).
 constexpr int kMaxDynamicSmem = 232448;
 
-// Launches fg8_gemm_kernel<BN> (sets its shared-memory limit on first use per
-// device).  Defined in the gemm_bn_*.cu instantiation files.
-template <int BN>
+// Launches fg8_gemm_kernel<BN, PAIR> on `grid` CTAs (PAIR: clusters of two).
+// On first use per device it checks the build's register count (the in-kernel
+// register split is safe only at exactly REGS_LAUNCH) and raises the kernel's
+// shared-memory limit.  Defined in gemm_inst.cu, one block width per object.
+template <int BN, bool PAIR>
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p, int grid,
                         size_t smem_bytes, cudaStream_t stream);
 
-template <int BN>
-int gemm_stage_bytes() {
-    return GemmShape<BN>::STAGE_BYTES;
+template <int BN, bool PAIR>
+cudaError_t launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p, int grid,
+                             size_t smem_bytes, cudaStream_t stream) {
+    static std::atomic<unsigned long long> attr_set{0};
+    static std::atomic<int> max_clusters[64];   // per device, 0 = not queried yet
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    auto kernel = fg8_gemm_kernel<BN, PAIR>;
+    if (!(attr_set.load() & bit)) {
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kernel);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != REGS_LAUNCH) return cudaErrorInvalidDeviceFunction;
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynamicSmem);
+        if (e != cudaSuccess) return e;
+        attr_set.fetch_or(bit);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // A persistent grid must fit on the device at once: clusters that do not
+        // would start only after others finish.  Query (once per device, at the
+        // largest shared-memory size, which all launches stay within) how many
+        // CTA pairs can be resident.
+        int mc = max_clusters[dev & 63].load();
+        if (mc == 0) {
+            cudaLaunchConfig_t q = cfg;
+            q.dynamicSmemBytes = kMaxDynamicSmem;
+            e = cudaOccupancyMaxActiveClusters(&mc, kernel, &q);
+            if (e != cudaSuccess) return e;
+            if (mc <= 0) return cudaErrorInvalidConfiguration;
+            max_clusters[dev & 63].store(mc);
+        }
+        if (grid > 2 * mc) cfg.gridDim.x = static_cast<unsigned>(2 * mc);
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, p);
 }
 
-#define FG8_DEFINE_LAUNCH(BN)                                                                                  \
+#define FG8_DEFINE_LAUNCH_ONE(BN, PAIR)                                                                        \
     template <>                                                                                                \
-    cudaError_t launch_gemm<BN>(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p, int grid, \
-                                size_t smem_bytes, cudaStream_t stream) {                                      \
-        static std::atomic<unsigned long long> attr_set{0};                                                    \
-        int dev = 0;                                                                                           \
-        cudaError_t e = cudaGetDevice(&dev);                                                                   \
-        if (e != cudaSuccess) return e;                                                                        \
-        const unsigned long long bit = 1ull << (dev & 63);                                                     \
-        if (!(attr_set.load() & bit)) {                                                                        \
-            /* The in-kernel register split is only safe at exactly REGS_LAUNCH. */                            \
-            cudaFuncAttributes fa;                                                                             \
-            e = cudaFuncGetAttributes(&fa, fg8_gemm_kernel<BN>);                                               \
-            if (e != cudaSuccess) return e;                                                                    \
-            if (fa.numRegs != REGS_LAUNCH) return cudaErrorInvalidDeviceFunction;                              \
-            e = cudaFuncSetAttribute(fg8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,         \
-                                     kMaxDynamicSmem);                                                         \
-            if (e != cudaSuccess) return e;                                                                    \
-            attr_set.fetch_or(bit);                                                                            \
-        }                                                                                                      \
-        fg8_gemm_kernel<BN><<<grid, NUM_THREADS, smem_bytes, stream>>>(tmA, tmB, p);                           \
-        return cudaGetLastError();                                                                             \
+    cudaError_t launch_gemm<BN, PAIR>(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,     \
+                                      int grid, size_t smem_bytes, cudaStream_t stream) {                      \
+        return launch_gemm_impl<BN, PAIR>(tmA, tmB, p, grid, smem_bytes, stream);                              \
     }
 
-#define FG8_DECLARE_LAUNCH(BN)                                                                                 \
+#define FG8_DECLARE_LAUNCH_ONE(BN, PAIR)                                                                       \
     template <>                                                                                                \
-    cudaError_t launch_gemm<BN>(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p, int grid, \
-                                size_t smem_bytes, cudaStream_t stream);
+    cudaError_t launch_gemm<BN, PAIR>(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,     \
+                                      int grid, size_t smem_bytes, cudaStream_t stream);
 
+// Block widths 16..256; CTA pairs from 32 (each CTA loads at least 16 B rows).
 #define FG8_FOR_EACH_BN(X) \
     X(16) X(32) X(48) X(64) X(80) X(96) X(112) X(128) X(144) X(160) X(176) X(192) X(208) X(224) X(240) X(256)
 

@@ -154,7 +154,8 @@ fg_status fg_set_wait_limit_ns(unsigned long long ns);
 unsigned long long fg_get_wait_limit_ns(void);
 
 /* The block width (BLOCK_N) the normal GEMM would use for (M, N, K) with the
- * current SM budget, or 0 for an unsupported shape.  Diagnostics. */
+ * current SM budget, negated when the tile runs on a pair of CTAs (256-row
+ * tiles), or 0 for an unsupported shape.  Diagnostics. */
 int fg_query_block_n(int M, int N, int K);
 
 #ifdef __cplusplus

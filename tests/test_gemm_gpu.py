@@ -88,9 +88,13 @@ def test_normal_gemm_matches_oracle(fg, M, N, K):
     check(D.double().cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("pair", [0, 1])
 @pytest.mark.parametrize("bn", list(range(16, 257, 16)))
-def test_every_block_width_matches_oracle(fg, bn, monkeypatch):
+def test_every_block_width_matches_oracle(fg, bn, pair, monkeypatch):
+    if pair and bn < 32:
+        pytest.skip("CTA pairs start at block width 32")
     monkeypatch.setenv("FG_FORCE_BLOCK_N", str(bn))
+    monkeypatch.setenv("FG_FORCE_PAIR", str(pair))
     M, N, K = 300, 400, 384   # ragged M and N, several K blocks, tiles straddling scale blocks
     x = synth.normal_inputs(M, N, K, seed=synth.seed_for(0, 60) + bn)
     A, sfa, B, sfb = to_gpu_normal(fg, x)
@@ -100,9 +104,10 @@ def test_every_block_width_matches_oracle(fg, bn, monkeypatch):
     check(D.double().cpu().numpy(), ref)
 
 
-@pytest.mark.parametrize("bn", [16, 112, 256])
-def test_permutation_b_is_bit_exact(fg, bn, monkeypatch):
+@pytest.mark.parametrize("bn,pair", [(16, 0), (112, 0), (256, 0), (32, 1), (112, 1), (256, 1)])
+def test_permutation_b_is_bit_exact(fg, bn, pair, monkeypatch):
     monkeypatch.setenv("FG_FORCE_BLOCK_N", str(bn))
+    monkeypatch.setenv("FG_FORCE_PAIR", str(pair))
     M, K = 130, 384
     N = K
     rng = np.random.default_rng(3)
@@ -189,13 +194,17 @@ def check_contiguous(fg, x, D, rows=None):
     check(Dc[torch.from_numpy(np.asarray(rows))].double().numpy(), ref)
 
 
-def test_contiguous_small(fg):
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_contiguous_small(fg, pair, monkeypatch):
+    monkeypatch.setenv("FG_FORCE_PAIR", pair)
     x = synth.contiguous_inputs(4, 272, 512, seed=synth.seed_for(2, 50), counts=[5, 0, 130, 256])
     D = run_contiguous(fg, x)
     check_contiguous(fg, x, D)
 
 
-def test_contiguous_all_padding_block_is_skipped(fg):
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_contiguous_all_padding_block_is_skipped(fg, pair, monkeypatch):
+    monkeypatch.setenv("FG_FORCE_PAIR", pair)
     x = synth.contiguous_inputs(2, 128, 256, seed=synth.seed_for(2, 51), counts=[100, 40])
     # add an all-padding block between the experts
     mi = x.m_indices.numpy()
@@ -235,13 +244,17 @@ def check_masked(fg, x, D, sample=None):
     check(flat[torch.from_numpy(rows)].double().numpy(), ref)
 
 
-def test_masked_small(fg):
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_masked_small(fg, pair, monkeypatch):
+    monkeypatch.setenv("FG_FORCE_PAIR", pair)
     x = synth.masked_inputs(5, 200, 144, 384, seed=synth.seed_for(3, 50), masked=[0, 1, 128, 200, 250])
     D = run_masked(fg, x)
     check_masked(fg, x, D)
 
 
-def test_masked_all_empty(fg):
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_masked_all_empty(fg, pair, monkeypatch):
+    monkeypatch.setenv("FG_FORCE_PAIR", pair)
     x = synth.masked_inputs(3, 64, 64, 128, seed=synth.seed_for(3, 51), masked=[0, 0, -5])
     D = run_masked(fg, x)
     check_masked(fg, x, D)
