@@ -3,8 +3,9 @@
     python -m fp8_fine_grained_tma_b200.build [--force] [--jobs N] [--verbose]
 
 Each GEMM block width (16..256 in steps of 16) is one object compiled from
-csrc/gemm_inst.cu with -DFG8_BN=<width>, in parallel; the host code is
-csrc/fg8_host.cu.  The CUDA runtime is linked statically, so the library
+csrc/gemm_inst.cu with -DFG8_BN=<width>, and each decode token-tile width
+(32..256 in steps of 32) one object from csrc/decode_inst.cu with
+-DFG8_MT=<width>, all in parallel; the host code is csrc/fg8_host.cu.  The CUDA runtime is linked statically, so the library
 needs only the NVIDIA driver at run time.
 """
 from __future__ import annotations
@@ -24,6 +25,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfg8.so")
 BLOCK_NS = list(range(16, 257, 16))
+DECODE_MTS = list(range(32, 257, 32))
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
 
@@ -65,6 +67,11 @@ def build(force: bool = False, jobs: int = 0, verbose: bool = False) -> str:
         objs.append(o)
         cmds.append([nvcc(), *ARCH, *FLAGS, *ptxas, f"-DFG8_BN={bn}", "-c",
                      os.path.join(CSRC, "gemm_inst.cu"), "-o", o])
+    for mt in DECODE_MTS:
+        o = os.path.join(BUILD, f"decode_mt_{mt}.o")
+        objs.append(o)
+        cmds.append([nvcc(), *ARCH, *FLAGS, *ptxas, f"-DFG8_MT={mt}", "-c",
+                     os.path.join(CSRC, "decode_inst.cu"), "-o", o])
     for src in ["fg8_host.cu"]:
         o = os.path.join(BUILD, src.replace(".cu", ".o"))
         objs.append(o)

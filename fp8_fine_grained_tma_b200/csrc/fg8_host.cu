@@ -13,6 +13,7 @@
 #include <mutex>
 #include <tuple>
 
+#include "decode_launch.cuh"
 #include "fg8.h"
 #include "launch.cuh"
 
@@ -21,6 +22,7 @@ namespace fg8 {
 #define FG8_DECLARE_BOTH(BN) FG8_DECLARE_LAUNCH_ONE(BN, false) FG8_DECLARE_LAUNCH_ONE(BN, true)
 FG8_FOR_EACH_BN(FG8_DECLARE_BOTH)
 #undef FG8_DECLARE_BOTH
+FG8_FOR_EACH_MT(FG8_DECLARE_DECODE_LAUNCH)
 
 // First error recorded by any GEMM kernel on this device: [0] = code,
 // [1] = (block << 8) | role.  Cleared by fg_get_last_device_status.
@@ -265,6 +267,235 @@ bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 
 constexpr long long kMaxDim = (1ll << 31) - 1;
 
+// ---- decode (few rows of A): split-K workspace ----------------------------------
+// One FP32 partial buffer and one counter array per (device, stream), grown on
+// demand and kept for the life of the process; launches on one stream run in
+// order, so they never share a buffer concurrently.  Counters are zero between
+// launches (each resets itself at its tile's last arrival); after a device-side
+// abort fg_get_last_device_status clears them.
+struct Workspace {
+    float* partials = nullptr;
+    size_t partial_bytes = 0;
+    unsigned* counters = nullptr;
+    size_t counter_count = 0;
+};
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+std::mutex g_ws_mutex;
+
+fg_status get_workspace(int dev, cudaStream_t stream, size_t partial_bytes, size_t counters, float** part,
+                        unsigned** ctr) {
+    std::lock_guard<std::mutex> lk(g_ws_mutex);
+    Workspace& w = g_ws[std::make_pair(dev, stream)];
+    if (w.partial_bytes < partial_bytes) {
+        if (w.partials) cudaFree(w.partials);
+        w.partials = nullptr;
+        w.partial_bytes = 0;
+        const size_t want = std::max(partial_bytes, 2 * w.partial_bytes);
+        if (cudaMalloc(&w.partials, want) != cudaSuccess) {
+            cudaGetLastError();
+            return FG_ERR_CUDA;
+        }
+        w.partial_bytes = want;
+    }
+    if (w.counter_count < counters) {
+        if (w.counters) cudaFree(w.counters);
+        w.counters = nullptr;
+        w.counter_count = 0;
+        const size_t want = std::max<size_t>(counters, 1024);
+        if (cudaMalloc(&w.counters, want * sizeof(unsigned)) != cudaSuccess ||
+            cudaMemset(w.counters, 0, want * sizeof(unsigned)) != cudaSuccess) {
+            cudaGetLastError();
+            return FG_ERR_CUDA;
+        }
+        w.counter_count = want;
+    }
+    *part = w.partials;
+    *ctr = w.counters;
+    return FG_OK;
+}
+
+// After an aborted launch some counters may hold a partial count: clear all of
+// this device's counters (synchronously; the caller has synchronised).
+void clear_workspace_counters(int dev) {
+    std::lock_guard<std::mutex> lk(g_ws_mutex);
+    for (auto& kv : g_ws)
+        if (kv.first.first == dev && kv.second.counters)
+            cudaMemset(kv.second.counters, 0, kv.second.counter_count * sizeof(unsigned));
+}
+
+int decode_tile_width(int M) { return std::max(32, (M + 31) / 32 * 32); }
+
+int decode_nbuf(int mt) { return std::min(DEC_MAX_NBUF, 512 / mt); }
+
+int decode_stages(int mt) {
+    const int sb = BM * BK + mt * BK;
+    int s = 8;
+    while (s > 2 && decode_smem_bytes(sb, s, mt) > static_cast<size_t>(kMaxDynamicSmem)) --s;
+    return s;
+}
+
+// Resident CTAs of fg8_decode_kernel<mt> when grouped in clusters of s
+// (cached per device; 0 when clusters of that size cannot be launched).
+int decode_cluster_slots(int dev, int mt, int s, size_t smem) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int>, int> cache;
+    const auto key = std::make_tuple(dev, mt, s);
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) return it->second;
+    }
+    int mc = 0;
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (mt) {
+#define FG8_DCAP(MTV) \
+    case MTV:         \
+        e = decode_max_clusters<MTV>(s, smem, &mc); \
+        break;
+        FG8_FOR_EACH_MT(FG8_DCAP)
+#undef FG8_DCAP
+        default:
+            break;
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        mc = 0;
+    }
+    const int slots = std::max(0, mc) * s;
+    std::lock_guard<std::mutex> lk(mu);
+    cache[key] = slots;
+    return slots;
+}
+
+struct DecodePlan {
+    int splits;
+    int cluster;   // 1, or == splits when the splits of a tile form one cluster
+};
+
+// Splits of K per 128-row tile of B, and whether they reduce inside a cluster.
+// Minimises the modelled time
+//   max(B bytes / HBM rate, waves * K blocks per split * t_kb) + waves * t_unit
+// with t_kb = 16 KiB / 64 GB/s (one SM streaming B alone), HBM rate 6.5 TB/s
+// and t_unit the pipeline ramp plus the split reduction: 1.5 us through the
+// global workspace (persistent grid), 1.0 us through distributed shared memory
+// (2..8 splits, every tile's cluster resident at once).
+DecodePlan decode_plan(int dev, int mt, size_t smem, int stage_room, int N, int K, int num_sms) {
+    const int KB = K / BK;
+    const int NB = (N + BM - 1) / BM;
+    const char* cenv = std::getenv("FG_DECODE_CLUSTER");
+    const bool cluster_ok = !(cenv && std::atoi(cenv) == 0) && stage_room >= mt * BM * 4;
+    auto cluster_fits = [&](int s) {
+        if (!cluster_ok || s < 2 || s > DEC_MAX_CLUSTER) return false;
+        const long long units = static_cast<long long>(NB) * s;
+        return units <= std::min(num_sms, decode_cluster_slots(dev, mt, s, smem));
+    };
+    const char* force = std::getenv("FG_FORCE_SPLITS");
+    if (force && std::atoi(force) >= 1) {
+        const int f = std::min(std::atoi(force), KB);
+        return DecodePlan{f, cluster_fits(f) ? f : 1};
+    }
+    const double t_hbm = static_cast<double>(N) * K / 6.5e12;
+    const double t_kb = 16384.0 / 64e9;
+    DecodePlan best{1, 1};
+    double best_t = 1e300;
+    for (int s = 1; s <= std::min(KB, 32); ++s) {
+        const int per = (KB + s - 1) / s;
+        const int used = (KB + per - 1) / per;   // splits that get work
+        if (used != s) continue;
+        const long long units = static_cast<long long>(NB) * s;
+        const double waves = static_cast<double>((units + num_sms - 1) / num_sms);
+        double t = std::max(t_hbm, waves * per * t_kb) + waves * 1.5e-6;
+        int cl = 1;
+        if (cluster_fits(s)) {
+            const double tc = std::max(t_hbm, per * t_kb) + 1.0e-6;
+            if (tc < t) {
+                t = tc;
+                cl = s;
+            }
+        }
+        if (t < best_t * 0.98) {
+            best_t = t;
+            best = DecodePlan{s, cl};
+        }
+    }
+    return best;
+}
+
+fg_status launch_decode_mt(int mt, const CUtensorMap& ta, const CUtensorMap& tb, const DecodeParams& p, int grid,
+                           int cluster, size_t smem, cudaStream_t st) {
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (mt) {
+#define FG8_DCASE(MTV) \
+    case MTV:          \
+        e = launch_decode<MTV>(ta, tb, p, grid, cluster, smem, st); \
+        break;
+        FG8_FOR_EACH_MT(FG8_DCASE)
+#undef FG8_DCASE
+        default:
+            return FG_ERR_UNSUPPORTED;
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return FG_ERR_CUDA;
+    }
+    return FG_OK;
+}
+
+fg_status run_decode(const void* A, const float* sfa, const void* B, const float* sfb, void* D, int M, int N, int K,
+                     cudaStream_t stream) {
+    DeviceInfo* dev = nullptr;
+    fg_status st = current_device(&dev);
+    if (st != FG_OK) return st;
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    const int num_sms = effective_sms(*dev);
+    const int mt = decode_tile_width(M);
+    const int stages = decode_stages(mt);
+    if (stages < decode_nbuf(mt)) return FG_ERR_UNSUPPORTED;   // the issuers' barrier invariant needs it
+    const int stage_bytes = BM * BK + mt * BK;
+    const size_t smem = decode_smem_bytes(stage_bytes, stages, mt);
+    const DecodePlan plan = decode_plan(dev_id, mt, smem, stages * stage_bytes, N, K, num_sms);
+
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.KB = K / BK;
+    p.NB = (N + BM - 1) / BM;
+    p.splits = plan.splits;
+    p.kb_per_split = (p.KB + p.splits - 1) / p.splits;
+    p.units = p.NB * p.splits;
+    p.cluster_reduce = plan.cluster > 1 ? 1 : 0;
+    p.stages = stages;
+    p.sfa_ld = static_cast<int>(fg_get_tma_aligned_size(M, 4));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.D = static_cast<__nv_bfloat16*>(D);
+    p.status = dev->status;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    if (p.splits > 1 && !p.cluster_reduce) {
+        st = get_workspace(dev_id, stream, static_cast<size_t>(p.units) * mt * BM * sizeof(float), p.NB,
+                           &p.workspace, &p.counters);
+        if (st != FG_OK) return st;
+    }
+    CUtensorMap ta, tb;
+    st = operand_map(A, K, M, 1, mt, &ta);
+    if (st != FG_OK) return st;
+    st = operand_map(B, K, N, 1, BM, &tb);
+    if (st != FG_OK) return st;
+    // Cluster mode: one CTA per unit (the whole grid is resident by the plan);
+    // otherwise a persistent grid.
+    const int grid = p.cluster_reduce ? p.units : std::max(1, std::min(p.units, num_sms));
+    return launch_decode_mt(mt, ta, tb, p, grid, plan.cluster, smem, stream);
+}
+
+// Rows of A up to which the normal GEMM uses the decode kernel.
+int decode_max_rows() {
+    const char* env = std::getenv("FG_DECODE_MAX_M");
+    return env ? std::atoi(env) : 128;
+}
+
 // Shared by the three GEMM kinds once their arguments are checked.
 fg_status run_gemm(int layout, const void* A, const float* sfa, const void* B, const float* sfb, void* D,
                    const int* m_indices, const int* masked_m, int rows, int N, int K, int G, int valid_rows_hint,
@@ -378,6 +609,8 @@ fg_status fg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const f
     if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sfa) || !aligned4(sfb))
         return FG_ERR_ALIGNMENT;
     if (static_cast<long long>(M) * N > kMaxDim * 4 || M > kMaxDim - 128) return FG_ERR_UNSUPPORTED;
+    if (M <= std::min(decode_max_rows(), 256))
+        return run_decode(A, sfa, B, sfb, D, M, N, K, reinterpret_cast<cudaStream_t>(stream));
     return run_gemm(LAYOUT_NORMAL, A, sfa, B, sfb, D, nullptr, nullptr, M, N, K, 1, M,
                     reinterpret_cast<cudaStream_t>(stream));
 }
@@ -479,6 +712,11 @@ fg_status fg_get_last_device_status(fg_stream_t stream, int* code_out, int* deta
     }
     *code_out = h[0];
     if (detail_out) *detail_out = h[1];
+    if (h[0] != 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        clear_workspace_counters(dev);
+    }
     return FG_OK;
 }
 

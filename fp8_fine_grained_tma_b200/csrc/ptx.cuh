@@ -260,6 +260,16 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
     return r;
 }
 
+// Load 16 bytes from the cluster shared window (possibly a peer CTA's memory).
+__device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(cluster_addr)
+                 : "memory");
+    return v;
+}
+
 // Arrive on an mbarrier given by its cluster-window address (possibly in the
 // peer CTA), with the default release semantics at CTA scope.  (An explicit
 // cluster-scope release fence here costs about 2000 cycles per arrival.)
@@ -313,6 +323,22 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask
             smem_addr(bar)),
         "h"(cta_mask)
         : "memory");
+}
+
+// Atomic increment with acquire-release semantics at GPU scope: wraps to 0
+// after reaching `limit` (so a counter of `limit + 1` arrivals resets itself).
+// Returns the old value.  The release half orders this thread's earlier writes
+// (and, through a preceding CTA barrier, those of the whole CTA) before the
+// increment; the acquire half orders later reads after it.
+__device__ __forceinline__ unsigned atom_inc_acq_rel_gpu(unsigned* addr, unsigned limit) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(limit) : "memory");
+    return old;
+}
+
+// Named barrier among `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Register reallocation across a warpgroup (all four warps must execute it).

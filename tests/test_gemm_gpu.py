@@ -318,3 +318,84 @@ def test_decode_sweep_sampled_rows(fg, si, M, N, K):
     rows = sample_rows(M, 8, si)
     ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), rows=rows)
     check(D[torch.from_numpy(rows).cuda()].double().cpu().numpy(), ref)
+
+
+# ------------------------------------------------------------ decode kernel --
+
+@pytest.mark.parametrize("splits,reduce", [("1", "any"), ("3", "cluster"), ("3", "workspace"),
+                                           ("5", "cluster"), ("5", "workspace"),
+                                           ("8", "cluster"), ("8", "workspace")])
+@pytest.mark.parametrize("M", [1, 17, 32, 64, 96, 100, 128, 160, 200, 256])
+def test_decode_kernel_matches_oracle(fg, M, splits, reduce, monkeypatch):
+    """Few rows of A: weights on the tensor core's 128-row side, K split over
+    CTAs and reduced in split order, inside a cluster through distributed
+    shared memory or through the global workspace; every token-tile width
+    32..256.  Five splits of 8 K blocks leave the last split empty."""
+    monkeypatch.setenv("FG_DECODE_MAX_M", "256")
+    monkeypatch.setenv("FG_FORCE_SPLITS", splits)
+    monkeypatch.setenv("FG_DECODE_CLUSTER", "0" if reduce == "workspace" else "1")
+    N, K = 400, 1024
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(4, 50) + M)
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    D = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    check(D.double().cpu().numpy(), ref)
+
+
+def test_decode_repeated_and_interleaved_launches(fg, monkeypatch):
+    """Split-K counters carry a launch epoch: back-to-back launches of
+    different shapes on one stream must each reduce correctly."""
+    monkeypatch.setenv("FG_FORCE_SPLITS", "5")
+    xs = [synth.normal_inputs(64, 2112, 1280, seed=synth.seed_for(4, 60)),
+          synth.normal_inputs(48, 1024, 2560, seed=synth.seed_for(4, 61))]
+    dev = [to_gpu_normal(fg, x) for x in xs]
+    outs = []
+    for _ in range(3):
+        for (A, sfa, B, sfb) in dev:
+            outs.append(fg.fp8_gemm_nt(A, sfa, B, sfb))
+    torch.cuda.synchronize()
+    refs = [oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy()) for x in xs]
+    for i, o in enumerate(outs):
+        check(o.double().cpu().numpy(), refs[i % 2])
+        assert torch.equal(o, outs[i % 2])   # deterministic reduction order
+
+
+def test_decode_more_splits_than_a_cluster(fg, monkeypatch):
+    """Above 8 splits the reduction always goes through the global workspace."""
+    monkeypatch.setenv("FG_FORCE_SPLITS", "12")
+    x = synth.normal_inputs(40, 528, 3072, seed=synth.seed_for(4, 64))
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    D = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    check(D.double().cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("M,N,K,splits", [(64, 2112, 7168, "8"), (128, 4096, 7168, "4"), (5, 768, 2048, "2")])
+def test_decode_cluster_and_workspace_reductions_agree(fg, M, N, K, splits, monkeypatch):
+    """Both split-K reductions add the splits in the same order, so their
+    results are equal element for element."""
+    monkeypatch.setenv("FG_FORCE_SPLITS", splits)
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(4, 63) + M)
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    monkeypatch.setenv("FG_DECODE_CLUSTER", "1")
+    D1 = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    monkeypatch.setenv("FG_DECODE_CLUSTER", "0")
+    D2 = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    assert torch.equal(D1, D2)
+    rows = sample_rows(M, 8, M)
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), rows=rows)
+    check(D1[torch.from_numpy(rows).cuda()].double().cpu().numpy(), ref)
+
+
+def test_small_m_on_the_tile_kernel(fg, monkeypatch):
+    """The 128-row tile kernel still handles few rows when the decode kernel is off."""
+    monkeypatch.setenv("FG_DECODE_MAX_M", "0")
+    x = synth.normal_inputs(64, 2112, 1024, seed=synth.seed_for(4, 62))
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    D = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    check(D.double().cpu().numpy(), ref)
