@@ -35,7 +35,7 @@ LIB_PATH = os.path.join(_HERE, "libfg8.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m fp8_fine_grained_tma_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python fp8_fine_grained_tma_b200/build.py` "
         "(there is no CPU fallback)")
 
 _lib = ctypes.CDLL(LIB_PATH)

@@ -13,7 +13,12 @@ HEADER = os.path.join(ROOT, "include", "fg8.h")
 
 @pytest.fixture(scope="module")
 def lib():
-    from fp8_fine_grained_tma_b200 import build
+    # build.py is loaded by path: importing the package needs the library.
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("fg8_build", os.path.join(ROOT, "fp8_fine_grained_tma_b200",
+                                                                            "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
     path = build.build()
     return ctypes.CDLL(path)
 
