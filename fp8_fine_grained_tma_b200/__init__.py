@@ -57,6 +57,7 @@ _SIG = {
     "fg_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
     "fg_get_wait_limit_ns": (ctypes.c_ulonglong, []),
     "fg_query_block_n": (_I, [_I, _I, _I]),
+    "fg_fp8_gemm_nt_small_m_no_alloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -188,6 +189,34 @@ def fp8_gemm_nt(A, sfa, B, sfb, D=None, stream=None):
     with torch.cuda.device(A.device):
         _check(_lib.fg_fp8_gemm_nt(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), M, N, K, _stream(stream)),
                "fp8_gemm_nt")
+    return D
+
+
+def fp8_gemm_nt_small_m_no_alloc(A, sfa, B, sfb, D, stream=None):
+    """fp8_gemm_nt for 1 <= M <= 256 that allocates no device memory: the
+    split-K scratch is a device array the library holds on every GPU it is
+    loaded on, so callers whose device memory is all reserved up front, or
+    that may not call cudaMalloc in their serving loop, can still split K.
+    D (bf16 [M, N]) must be given.  Calls that overlap on the GPU share that
+    scratch and race; the first call on a device, which looks up the scratch
+    address, should come before any stream capture."""
+    A = _codes(A, "A")
+    B = _codes(B, "B")
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K:
+        raise ValueError("A and B disagree on K")
+    KB = K // BLOCK
+    _check_sfa(sfa, None, M, KB)
+    _f32(sfb, "sfb")
+    if tuple(sfb.shape) != ((N + BLOCK - 1) // BLOCK, KB) or not sfb.is_contiguous():
+        raise ValueError(f"sfb must be contiguous [{(N + BLOCK - 1) // BLOCK}, {KB}]")
+    if D.dtype != torch.bfloat16 or tuple(D.shape) != (M, N) or not D.is_contiguous():
+        raise ValueError("D must be a contiguous bf16 [M, N] tensor")
+    with torch.cuda.device(A.device):
+        _check(_lib.fg_fp8_gemm_nt_small_m_no_alloc(_ptr(A), _ptr(sfa), _ptr(B), _ptr(sfb), _ptr(D), M, N, K,
+                                                    _stream(stream)),
+               "fp8_gemm_nt_small_m_no_alloc")
     return D
 
 

@@ -740,3 +740,129 @@ int fg_query_block_n(int M, int N, int K) {
 }
 
 }  // extern "C"
+
+// ---- few-rows GEMM on library-owned scratch (fg_fp8_gemm_nt_small_m_no_alloc) --
+namespace fg8 {
+
+// Split-K scratch of the no-allocation entry point, one copy per device:
+// [FG_NO_ALLOC_MAX_N / 128 arrival counters (unsigned)]
+// [FG_NO_ALLOC_PARTIAL_FLOATS partial sums (float)].
+// Host code must not use this name as an address; it takes the device address
+// from cudaGetSymbolAddress (no_alloc_scratch below).
+constexpr size_t kNoAllocCounterBytes = static_cast<size_t>(FG_NO_ALLOC_MAX_N / BM) * sizeof(unsigned);
+static_assert(kNoAllocCounterBytes % 256 == 0, "partials start 256-byte aligned");
+static __device__ __align__(256) unsigned char g_no_alloc_scratch[FG_NO_ALLOC_SCRATCH_BYTES];
+
+namespace {
+
+unsigned char* g_no_alloc_ptr[kMaxDevices];
+std::mutex g_no_alloc_mutex;
+
+// Device address of the scratch on device `dev` (current), looked up once.
+fg_status no_alloc_scratch(int dev, unsigned char** out) {
+    std::lock_guard<std::mutex> lk(g_no_alloc_mutex);
+    if (!g_no_alloc_ptr[dev]) {
+        void* addr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&addr, g_no_alloc_scratch);
+        if (e != cudaSuccess || !addr) {
+            cudaGetLastError();
+            return FG_ERR_CUDA;
+        }
+        g_no_alloc_ptr[dev] = static_cast<unsigned char*>(addr);
+    }
+    *out = g_no_alloc_ptr[dev];
+    return FG_OK;
+}
+
+// The operand descriptor of operand_map, encoded on the stack (no cache).
+fg_status operand_map_uncached(const void* ptr, uint64_t K, uint64_t rows, uint32_t box_rows, CUtensorMap* out) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return FG_ERR_NO_DEVICE;
+    std::memset(out, 0, sizeof(*out));
+    const cuuint64_t dims[3] = {K, rows, 1};
+    const cuuint64_t strides[2] = {K, K * rows};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FG_OK : FG_ERR_CUDA;
+}
+
+// The decode kernel in workspace mode with the scratch above as workspace.
+fg_status run_decode_no_alloc(const void* A, const float* sfa, const void* B, const float* sfb, void* D, int M,
+                              int N, int K, cudaStream_t stream) {
+    DeviceInfo* dev = nullptr;
+    fg_status st = current_device(&dev);
+    if (st != FG_OK) return st;
+    int dev_id = 0;
+    if (cudaGetDevice(&dev_id) != cudaSuccess) {
+        cudaGetLastError();
+        return FG_ERR_CUDA;
+    }
+    unsigned char* scratch = nullptr;
+    st = no_alloc_scratch(dev_id, &scratch);
+    if (st != FG_OK) return st;
+    const int num_sms = effective_sms(*dev);
+    const int mt = decode_tile_width(M);
+    const int stages = decode_stages(mt);
+    if (stages < decode_nbuf(mt)) return FG_ERR_UNSUPPORTED;
+    const size_t smem = decode_smem_bytes(BM * BK + mt * BK, stages, mt);
+    // No room for cluster staging: the plan picks the workspace reduction.
+    DecodePlan plan = decode_plan(dev_id, mt, smem, 0, N, K, num_sms);
+    const int KB = K / BK;
+    const int NB = (N + BM - 1) / BM;
+    int splits = plan.splits;
+    while (splits > 1 && static_cast<size_t>(NB) * splits * mt * BM > FG_NO_ALLOC_PARTIAL_FLOATS) --splits;
+
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.KB = KB;
+    p.NB = NB;
+    p.splits = splits;
+    p.kb_per_split = (KB + splits - 1) / splits;
+    p.units = NB * splits;
+    p.cluster_reduce = 0;
+    p.stages = stages;
+    p.sfa_ld = static_cast<int>(fg_get_tma_aligned_size(M, 4));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.D = static_cast<__nv_bfloat16*>(D);
+    p.status = dev->status;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    if (splits > 1) {
+        p.counters = reinterpret_cast<unsigned*>(scratch);
+        p.workspace = reinterpret_cast<float*>(scratch + kNoAllocCounterBytes);
+        // The counters must start at zero; an earlier call may have left any value.
+        if (cudaMemsetAsync(p.counters, 0, static_cast<size_t>(NB) * sizeof(unsigned), stream) != cudaSuccess) {
+            cudaGetLastError();
+            return FG_ERR_CUDA;
+        }
+    }
+    CUtensorMap ta, tb;
+    st = operand_map_uncached(A, K, M, mt, &ta);
+    if (st != FG_OK) return st;
+    st = operand_map_uncached(B, K, N, BM, &tb);
+    if (st != FG_OK) return st;
+    const int grid = std::max(1, std::min(p.units, num_sms));
+    return launch_decode_mt(mt, ta, tb, p, grid, 1, smem, stream);
+}
+
+}  // namespace
+}  // namespace fg8
+
+extern "C" fg_status fg_fp8_gemm_nt_small_m_no_alloc(const void* A, const float* sfa, const void* B,
+                                                     const float* sfb, void* D, int M, int N, int K,
+                                                     fg_stream_t stream) {
+    if (M < 0 || N < 0 || K < 0) return FG_ERR_INVALID_ARG;
+    if (K == 0 || K % 128 != 0 || N % 16 != 0) return FG_ERR_UNSUPPORTED;
+    if (M > FG_NO_ALLOC_MAX_M || N > FG_NO_ALLOC_MAX_N) return FG_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return FG_OK;
+    if (!A || !sfa || !B || !sfb || !D) return FG_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sfa) || !aligned4(sfb))
+        return FG_ERR_ALIGNMENT;
+    return run_decode_no_alloc(A, sfa, B, sfb, D, M, N, K, reinterpret_cast<cudaStream_t>(stream));
+}

@@ -158,6 +158,49 @@ unsigned long long fg_get_wait_limit_ns(void);
  * tiles), or 0 for an unsupported shape.  Diagnostics. */
 int fg_query_block_n(int M, int N, int K);
 
+/*
+ * Few-rows normal GEMM that allocates nothing.  The pages have no counterpart
+ * to this entry point: it is an addition of this library.
+ *
+ * Why: fg_fp8_gemm_nt, when it splits K over several CTAs for a small M, may
+ * call cudaMalloc the first time it needs its split-K workspace on a device
+ * and stream (or a larger one).  Some callers cannot let that happen: a
+ * serving engine that reserved nearly all device memory for its own pool
+ * up front (the allocation would fail), or a latency-critical loop in which
+ * cudaMalloc / cudaFree, which may synchronise the device, are not allowed.
+ * This entry point computes the same result as fg_fp8_gemm_nt, with the same
+ * operands, layouts and alignment rules, but keeps its split-K partial sums
+ * and arrival counters in a scratch array that the library defines as a
+ * device variable: every GPU that loads the library holds one copy of it
+ * (FG_NO_ALLOC_SCRATCH_BYTES) from module load until the process exits.  It
+ * never calls cudaMalloc, cudaFree or any allocating routine; the caller
+ * passes every input and output.  (Under CUDA's default lazy module loading
+ * the driver places a kernel's code in device memory at its first launch; a
+ * caller that must avoid even that at run time makes one call per shape
+ * class first, or sets CUDA_MODULE_LOADING=EAGER.)
+ *
+ * Limits: 1 <= M <= FG_NO_ALLOC_MAX_M and N <= FG_NO_ALLOC_MAX_N; larger sizes
+ * return FG_ERR_UNSUPPORTED and launch nothing.  The K split count is lowered
+ * until the partial sums fit in FG_NO_ALLOC_PARTIAL_FLOATS floats (one split
+ * needs no scratch).  M == 0 is a no-op.
+ *
+ * First call on a device: it looks up the scratch array's device address
+ * (cudaGetSymbolAddress) with that device current, once per device; make
+ * that first call before any stream capture.
+ *
+ * Sharing: every call on a device uses the same scratch and leaves its
+ * contents behind (each call clears the counters it needs on `stream` before
+ * its kernel runs).  Calls whose executions overlap on the GPU (other streams,
+ * other host threads) race on the scratch and may return wrong results:
+ * order them, e.g. on one stream.
+ */
+#define FG_NO_ALLOC_MAX_M 256
+#define FG_NO_ALLOC_MAX_N 262144
+#define FG_NO_ALLOC_PARTIAL_FLOATS (2u * 1024u * 1024u)
+#define FG_NO_ALLOC_SCRATCH_BYTES ((FG_NO_ALLOC_MAX_N / 128) * 4u + FG_NO_ALLOC_PARTIAL_FLOATS * 4u)
+fg_status fg_fp8_gemm_nt_small_m_no_alloc(const void* A, const float* sfa, const void* B, const float* sfb, void* D,
+                                          int M, int N, int K, fg_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -50,7 +50,8 @@ def test_binding_exposes_same_names():
         if py in ("status_string", "version", "get_last_device_status", "set_wait_limit_ns",
                   "get_wait_limit_ns", "query_block_n", "get_num_sms", "set_num_sms",
                   "get_m_alignment_for_contiguous_layout", "get_tma_aligned_size",
-                  "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked"):
+                  "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
+                  "fp8_gemm_nt_small_m_no_alloc"):
             assert hasattr(fg, py), py
     assert hasattr(fg, "get_col_major_tma_aligned_tensor")
 
@@ -104,6 +105,18 @@ def test_grouped_argument_checks(lib):
     assert m(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 40, 256, 0, None) == FG_ERR_UNSUPPORTED
     assert m(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 128, 256, -1, None) == FG_ERR_INVALID_ARG
     assert m(None, None, None, None, None, None, 0, 256, 128, 256, 0, None) == FG_OK  # no groups: no-op
+
+
+def test_no_alloc_argument_checks(lib):
+    f = lib.fg_fp8_gemm_nt_small_m_no_alloc
+    f.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+    f.restype = ctypes.c_int
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 257, 128, 256, None) == FG_ERR_UNSUPPORTED      # M above 256
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 262160, 256, None) == FG_ERR_UNSUPPORTED    # N above 262144
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 128, 200, None) == FG_ERR_UNSUPPORTED
+    assert f(FAKE + 8, FAKE, FAKE, FAKE, FAKE, 64, 128, 256, None) == FG_ERR_ALIGNMENT
+    assert f(None, FAKE, FAKE, FAKE, FAKE, 64, 128, 256, None) == FG_ERR_INVALID_ARG
+    assert f(None, None, None, None, None, 0, 128, 256, None) == FG_OK
 
 
 def test_helpers(lib):
