@@ -298,8 +298,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
         } else if (warp == DEC_SCALE_WARP) {
             // scol[m] = sfa[m, kb] * sfb[tile, kb] for every K block, in order.
-            // Loads run SCALE_AHEAD K blocks ahead of the writes, so the warp
-            // pays one global round trip per SCALE_AHEAD blocks, not per block.
+            // Loads run SCALE_AHEAD K blocks ahead of the writes.  The loop is
+            // unrolled by SCALE_AHEAD so that each register slot is refilled in
+            // place: a rotating copy would stall on the newest load every block.
             constexpr int SCALE_AHEAD = 4;
             constexpr int PER_LANE = MT / 32;
             DecodeCursor ld(p, blockIdx.x, gridDim.x);    // next (unit, K block) to load
@@ -314,27 +315,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int slot = 0;
             uint32_t sphase = 0;
             int w = 0;
-            while (wr.valid) {
-                if (lane == 0) w = wait_bar(&sempty[slot], sphase ^ 1u, limit, abort_flag);
-                w = __shfl_sync(0xffffffffu, w, 0);
-                if (w) break;
-                float* dst = scale_ring + slot * MT;
+            while (wr.valid && w == 0) {
 #pragma unroll
-                for (int i = 0; i < PER_LANE; ++i) dst[lane + 32 * i] = qa[0][i] * qb[0];
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&sfull[slot]);
+                for (int q = 0; q < SCALE_AHEAD; ++q) {
+                    if (!wr.valid) break;
+                    if (lane == 0) w = wait_bar(&sempty[slot], sphase ^ 1u, limit, abort_flag);
+                    w = __shfl_sync(0xffffffffu, w, 0);
+                    if (w) break;
+                    float* dst = scale_ring + slot * MT;
 #pragma unroll
-                for (int q = 0; q + 1 < SCALE_AHEAD; ++q) {
-#pragma unroll
-                    for (int i = 0; i < PER_LANE; ++i) qa[q][i] = qa[q + 1][i];
-                    qb[q] = qb[q + 1];
-                }
-                load_scales<MT>(p, ld, lane, qa[SCALE_AHEAD - 1], qb[SCALE_AHEAD - 1]);
-                ld.advance(p, gridDim.x);
-                wr.advance(p, gridDim.x);
-                if (++slot == DEC_SCALE_SLOTS) {
-                    slot = 0;
-                    sphase ^= 1u;
+                    for (int i = 0; i < PER_LANE; ++i) dst[lane + 32 * i] = qa[q][i] * qb[q];
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&sfull[slot]);
+                    load_scales<MT>(p, ld, lane, qa[q], qb[q]);
+                    ld.advance(p, gridDim.x);
+                    wr.advance(p, gridDim.x);
+                    if (++slot == DEC_SCALE_SLOTS) {
+                        slot = 0;
+                        sphase ^= 1u;
+                    }
                 }
             }
             if (w == 2 && lane == 0) record_error(p.status, ERR_TIMEOUT, ROLE_PRODUCER);
