@@ -5,9 +5,12 @@
 One step runs every GEMM of the workload once on inputs already resident in
 HBM.  The default workload is the prefill normal GEMM, M=4096 with (N,K) in
 {(24576,1536), (7168,16384), (4096,7168)}; the other workloads (decode,
-contiguous, masked, decode_sweep) are for profiling.  Each GEMM is timed with
-CUDA events on its launch stream after an L2 flush (a 512 MiB write), and
-``value`` = FLOPs of all timed GEMMs / their summed device time, in TFLOPS.
+contiguous, masked, decode_sweep) are for profiling.  Every GEMM keeps several
+copies of its operands, together larger than twice the L2 cache, and step s
+uses copy s mod copies, so no launch finds its operands in L2.  Each launch is
+timed with CUDA events on its launch stream; a short GPU spin before the start
+event absorbs the host's launch latency.  ``value`` = FLOPs of all timed GEMMs
+/ their summed device time, in TFLOPS.
 
 N > 1 (under torchrun): every rank runs the same workload on its own GPU
 (independent replicas, no collective on the data path; weak scaling); the
@@ -55,7 +58,9 @@ WORKLOADS = {
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0          # nominal dense ratio 4.5 / 2.25 PFLOP/s
-FLUSH_BYTES = 512 << 20
+L2_BYTES = 126 << 20
+MAX_COPIES = 32
+SPIN_CYCLES = 100_000        # ~50 us at 1.965 GHz: longer than one launch's host latency
 
 
 def load_peaks():
@@ -73,13 +78,32 @@ class Case:
     """One GEMM call of a workload: device inputs, its launcher, and its
     algorithmic FLOPs and HBM bytes."""
 
-    def __init__(self, name, flops, hbm_bytes, run, host=None):
+    def __init__(self, name, flops, hbm_bytes, run, host=None, copies=1):
         self.name = name
         self.flops = flops
         self.hbm_bytes = hbm_bytes
-        self.run = run
+        self.run = run            # run(i): one launch on operand copy i % copies
         self.host = host or {}
         self.block_n = None
+        self.copies = copies
+
+
+def n_copies(footprint_bytes):
+    """Operand copies whose total exceeds twice the L2 cache."""
+    return int(min(MAX_COPIES, max(1, -(-2 * L2_BYTES // max(1, footprint_bytes)))))
+
+
+def operand_copies(fg, x, D, n, extra=()):
+    """n operand sets for one GEMM (set 0 uses the originals): A, B, sfb, D and
+    the named extra tensors are cloned, sfa is laid out again from x.sfa."""
+    sets = []
+    for i in range(n):
+        t = {"A": x.A, "B": x.B, "sfb": x.sfb, "D": D, **{k: getattr(x, k) for k in extra}}
+        if i > 0:
+            t = {k: v.clone() for k, v in t.items()}
+        t["sfa"] = fg.get_col_major_tma_aligned_tensor(x.sfa)
+        sets.append(t)
+    return sets
 
 
 def ceil_div(a, b):
@@ -95,22 +119,22 @@ def build_cases(fg, synth, wl, device):
             for (N, K) in wl["shapes"]:
                 x = synth.normal_inputs(M, N, K, seed=synth.seed_for(wl["cfg"], si), device=device)
                 si += 1
-                sfa = fg.get_col_major_tma_aligned_tensor(x.sfa)
                 D = torch.empty((M, N), dtype=torch.bfloat16, device=device)
                 KB = K // 128
                 flops = 2.0 * M * N * K
                 hbm = M * K + N * K + M * KB * 4 + ceil_div(N, 128) * KB * 4 + 2 * M * N
+                sets = operand_copies(fg, x, D, n_copies(hbm))
 
-                def run(A=x.A, sfa=sfa, B=x.B, sfb=x.sfb, D=D):
-                    fg.fp8_gemm_nt(A, sfa, B, sfb, D=D)
+                def run(i, sets=sets):
+                    t = sets[i % len(sets)]
+                    fg.fp8_gemm_nt(t["A"], t["sfa"], t["B"], t["sfb"], D=t["D"])
 
-                c = Case(f"M{M}_N{N}_K{K}", flops, hbm, run, host={"x": x, "D": D})
+                c = Case(f"M{M}_N{N}_K{K}", flops, hbm, run, host={"x": x, "D": D}, copies=len(sets))
                 c.block_n = fg.query_block_n(M, N, K)
                 cases.append(c)
     elif kind == "contiguous":
         for si, (N, K) in enumerate(wl["shapes"]):
             x = synth.contiguous_inputs(wl["G"], N, K, seed=synth.seed_for(wl["cfg"], si), device=device)
-            sfa = fg.get_col_major_tma_aligned_tensor(x.sfa)
             D = torch.empty((x.M_tot, N), dtype=torch.bfloat16, device=device)
             real = sum(x.counts)
             KB = K // 128
@@ -118,16 +142,17 @@ def build_cases(fg, synth, wl, device):
             flops = 2.0 * real * N * K
             hbm = real * K + used * N * K + real * KB * 4 + used * ceil_div(N, 128) * KB * 4 + 2 * real * N \
                 + 4 * x.M_tot
+            sets = operand_copies(fg, x, D, n_copies(hbm), extra=("m_indices",))
 
-            def run(A=x.A, sfa=sfa, B=x.B, sfb=x.sfb, mi=x.m_indices, D=D):
-                fg.m_grouped_fp8_gemm_nt_contiguous(A, sfa, B, sfb, mi, D=D)
+            def run(i, sets=sets):
+                t = sets[i % len(sets)]
+                fg.m_grouped_fp8_gemm_nt_contiguous(t["A"], t["sfa"], t["B"], t["sfb"], t["m_indices"], D=t["D"])
 
             cases.append(Case(f"contig_G{wl['G']}_Mtot{x.M_tot}_N{N}_K{K}", flops, hbm, run,
-                              host={"x": x, "D": D}))
+                              host={"x": x, "D": D}, copies=len(sets)))
     elif kind == "masked":
         for si, (N, K) in enumerate(wl["shapes"]):
             x = synth.masked_inputs(wl["G"], wl["M_max"], N, K, seed=synth.seed_for(wl["cfg"], si), device=device)
-            sfa = fg.get_col_major_tma_aligned_tensor(x.sfa)
             D = torch.empty((x.G, x.M_max, N), dtype=torch.bfloat16, device=device)
             mm = [min(max(int(v), 0), x.M_max) for v in x.masked_m.cpu().tolist()]
             real = sum(mm)
@@ -135,12 +160,15 @@ def build_cases(fg, synth, wl, device):
             KB = K // 128
             flops = 2.0 * real * N * K
             hbm = real * K + used * N * K + real * KB * 4 + used * ceil_div(N, 128) * KB * 4 + 2 * real * N + 4 * x.G
+            sets = operand_copies(fg, x, D, n_copies(hbm), extra=("masked_m",))
 
-            def run(A=x.A, sfa=sfa, B=x.B, sfb=x.sfb, mm_t=x.masked_m, D=D):
-                fg.m_grouped_fp8_gemm_nt_masked(A, sfa, B, sfb, mm_t, expected_m=128, D=D)
+            def run(i, sets=sets):
+                t = sets[i % len(sets)]
+                fg.m_grouped_fp8_gemm_nt_masked(t["A"], t["sfa"], t["B"], t["sfb"], t["masked_m"], expected_m=128,
+                                                D=t["D"])
 
             cases.append(Case(f"masked_G{x.G}_Mmax{x.M_max}_N{N}_K{K}", flops, hbm, run,
-                              host={"x": x, "D": D, "masked": mm}))
+                              host={"x": x, "D": D, "masked": mm}, copies=len(sets)))
     return cases
 
 
@@ -265,7 +293,7 @@ def oracle_sample(cases, budget_s, rng_seed=0):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill")
@@ -303,20 +331,19 @@ def main(argv=None):
     cases = build_cases(fg, synth, wl, device)
     if args.case_index is not None:
         cases = [cases[args.case_index]]
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
-    def one_step(events=None):
+    def one_step(s, events=None):
         for ci, c in enumerate(cases):
-            flush.fill_(1.0)
+            torch.cuda._sleep(SPIN_CYCLES)    # the GPU idles here while the host enqueues the launch
             if events is not None:
                 events[ci][0].record(stream)
-            c.run()
+            c.run(s)
             if events is not None:
                 events[ci][1].record(stream)
 
-    for _ in range(args.warmup):
-        one_step()
+    for s in range(args.warmup):
+        one_step(s)
     torch.cuda.synchronize()
     code, detail = fg.get_last_device_status()
     if code != 0:
@@ -331,7 +358,7 @@ def main(argv=None):
     clocks.start()
     time.sleep(0.3)
     for s in range(args.steps):
-        one_step(evs[s])
+        one_step(args.warmup + s, evs[s])
     torch.cuda.synchronize()
     if pg is not None:
         pg.barrier()
@@ -397,7 +424,9 @@ def main(argv=None):
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate, bf16 out)",
         "data": "synthetic (seeded N(0,1), block-quantised to E4M3)",
         "config": {"workload": wl["desc"], "cases": [c.name for c in cases],
-                   "l2": "flushed before every GEMM (512 MiB write); only GEMM launches are timed",
+                   "l2": "inputs larger than L2: each GEMM rotates over operand copies totalling > 2 x 126 MB "
+                         "(copies per GEMM: " + ", ".join(str(c.copies) for c in cases) + "); only GEMM launches "
+                         "are timed (CUDA events around each launch, a GPU spin before each start event)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "per_shape": per_shape, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": len(cases) * args.steps, "clocks": clk, "impl": "ours",
@@ -472,18 +501,25 @@ def run_e2e(fg, cases, args, device, stream, pg, world):
 
 def read_traffic(workload):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, if it was taken on the current kernel source; else None."""
+    summary, if it was taken on the current source of that kernel; else None."""
     import hashlib
+    import re
     summ = os.path.join(ROOT, "profiles", f"ncu_traffic_{workload}.txt")
-    src = os.path.join(ROOT, "fp8_fine_grained_tma_b200", "csrc", "gemm_kernel.cuh")
     if not os.path.exists(summ):
         return None
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     vals = {}
     for line in open(summ):
-        if ":" in line:
-            k, v = line.split(":", 1)
-            vals[k.strip()] = v.strip()
+        if line.startswith("#") or ":" not in line:
+            continue
+        k, v = line.split(":", 1)
+        vals[k.strip()] = v.strip()
+    m = re.search(r"\((csrc/[\w.]+)\)", vals.get("kernel", ""))
+    if not m:
+        return None
+    src = os.path.join(ROOT, "fp8_fine_grained_tma_b200", m.group(1))
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     if vals.get("kernel_source_sha256_16") != h:
         return None
     try:
