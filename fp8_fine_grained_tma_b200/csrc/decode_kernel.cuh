@@ -351,15 +351,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t sphase = 0;
         bool ok = true;
         DecodeUnit d;
-        for (int u = blockIdx.x; ok && decode_unit(p, u, d); u += gridDim.x) {
-            // (ok turns false on an abort; the unit's epilogue barriers still run)
+        // Every promotion warp walks all of this CTA's units, even after an abort
+        // (ok turns false: the warp then skips the waits and the memory work), so
+        // all warps run the same sequence of named barriers in the split-K
+        // epilogue: warps that saw the abort in different units still meet there.
+        for (int u = blockIdx.x; decode_unit(p, u, d); u += gridDim.x) {
             float2 acc[CPW][8];
 #pragma unroll
             for (int i = 0; i < CPW; ++i)
 #pragma unroll
                 for (int q = 0; q < 8; ++q) acc[i][q] = make_float2(0.0f, 0.0f);
 
-            for (int kb = d.kb0; kb < d.kb1; ++kb) {
+            for (int kb = d.kb0; ok && kb < d.kb1; ++kb) {
                 int w = 0;
                 if (lane == 0) {
                     w = wait_bar(&tfull[buf], bphase, limit, abort_flag);

@@ -399,3 +399,47 @@ def test_small_m_on_the_tile_kernel(fg, monkeypatch):
     torch.cuda.synchronize()
     ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
     check(D.double().cpu().numpy(), ref)
+
+
+# ------------------------------------------------------ failure detection --
+
+FG_ERR_TIMEOUT = 6
+
+
+@pytest.mark.parametrize("M,N,K,env,sms", [(4096, 4096, 7168, {}, 0),
+                                           (64, 2112, 7168, {"FG_DECODE_CLUSTER": "0", "FG_FORCE_SPLITS": "8"}, 1)])
+def test_wait_timeout_is_reported_and_the_context_stays_usable(fg, monkeypatch, M, N, K, env, sms):
+    """With a 1 us limit on every pipeline wait, some wait of the GEMM runs
+    out: the kernel records FG_ERR_TIMEOUT, stops its roles, drains its
+    copies and returns.  The context must stay usable and the next call, with
+    the normal limit, must be correct (split-K counters left behind by the
+    abort are cleared when the status is read).  The decode case runs on one
+    SM, so that its MMA issuers wait for whole split-K epilogues and several
+    units pass through one CTA after the abort."""
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(4, 70) + M)
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    old = fg.get_wait_limit_ns()
+    old_sms = fg.get_num_sms()
+    codes = []
+    try:
+        if sms:
+            fg.set_num_sms(sms)
+        fg.set_wait_limit_ns(1000)
+        for _ in range(5):
+            fg.fp8_gemm_nt(A, sfa, B, sfb)
+            codes.append(fg.get_last_device_status()[0])
+            if codes[-1] == FG_ERR_TIMEOUT:
+                break
+    finally:
+        fg.set_wait_limit_ns(old)
+        fg.set_num_sms(old_sms)
+    assert FG_ERR_TIMEOUT in codes, codes
+    assert set(codes) <= {0, FG_ERR_TIMEOUT}
+    D = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    assert fg.get_last_device_status()[0] == 0
+    rows = sample_rows(M, 8, 70)
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), rows=rows)
+    check(D[torch.from_numpy(rows).cuda()].double().cpu().numpy(), ref)
