@@ -54,6 +54,9 @@ WORKLOADS = {
                      "shapes": [(2112, 7168), (24576, 1536), (32768, 512), (7168, 16384), (4096, 7168),
                                 (7168, 2048)],
                      "desc": "small-M decode sweep, M in {64,128} x 6 (N,K)"},
+    "quantize": {"kind": "quantize", "shapes": [(4096, 7168, "fp32"), (4096, 7168, "bf16"), (64, 7168, "bf16")],
+                 "desc": "activation quantiser (1x128 blocks -> E4M3 + MN-major FP32 scales), "
+                         "(M,K,dtype) in {(4096,7168,fp32),(4096,7168,bf16),(64,7168,bf16)}"},
 }
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -150,6 +153,20 @@ def build_cases(fg, synth, wl, device):
 
             cases.append(Case(f"contig_G{wl['G']}_Mtot{x.M_tot}_N{N}_K{K}", flops, hbm, run,
                               host={"x": x, "D": D}, copies=len(sets)))
+    elif kind == "quantize":
+        for si, (M, K, dt) in enumerate(wl["shapes"]):
+            g = torch.Generator(device=device)
+            g.manual_seed(synth.seed_for(5, si))
+            x = torch.randn((M, K), generator=g, device=device, dtype=torch.float32)
+            if dt == "bf16":
+                x = x.to(torch.bfloat16)
+            hbm = M * K * (x.element_size() + 1) + M * (K // 128) * 4
+            sets = [x] + [x.clone() for _ in range(n_copies(hbm) - 1)]
+
+            def run(i, sets=sets):
+                fg.quantize_fp8_activations(sets[i % len(sets)])
+
+            cases.append(Case(f"quant_M{M}_K{K}_{dt}", 0.0, hbm, run, host={"xq": x}, copies=len(sets)))
     elif kind == "masked":
         for si, (N, K) in enumerate(wl["shapes"]):
             x = synth.masked_inputs(wl["G"], wl["M_max"], N, K, seed=synth.seed_for(wl["cfg"], si), device=device)
@@ -377,9 +394,13 @@ def main(argv=None):
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
         total_ms = float(t.item())
     value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    unit = UNIT
+    if flops_step == 0:   # a bandwidth-bound workload (the quantiser): GB/s
+        value = world * sum(c.hbm_bytes for c in cases) * args.steps / (total_ms * 1e-3) / 1e9
+        unit = "GB/s"
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and wl["kind"] != "quantize":
         e2e = run_e2e(fg, cases, args, device, stream, pg, world)
 
     if rank != 0:
@@ -413,13 +434,26 @@ def main(argv=None):
                 "peak_source": f"{peak_src}: hbm_gbs (copy bandwidth)"}
 
     cpu = None
-    if not args.no_cpu_baseline and world == 1:
+    if not args.no_cpu_baseline and world == 1 and wl["kind"] == "quantize":
+        import oracle
+        c0 = cases[0]
+        xs = c0.host["xq"][:256].float().cpu().numpy()
+        t0 = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - t0 < args.cpu_budget_s:
+            oracle.quantize_blocks(xs, 1)
+            reps += 1
+        secs = time.perf_counter() - t0
+        cpu = {"value": round(reps * xs.shape[0] * xs.shape[1] * 5 / secs / 1e9, 4), "unit": "GB/s", "cores": 1,
+               "kind": "oracle", "sample": f"{reps} x quantize_blocks on 256 rows of {c0.name}",
+               "seconds": round(secs, 2)}
+    elif not args.no_cpu_baseline and world == 1:
         f, secs, thr, desc = oracle_sample(cases, args.cpu_budget_s)
         cpu = {"value": round(f / secs / 1e12, 6), "unit": UNIT, "cores": thr, "kind": "oracle", "sample": desc,
                "seconds": round(secs, 2)}
 
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate, bf16 out)",
         "data": "synthetic (seeded N(0,1), block-quantised to E4M3)",
@@ -534,6 +568,31 @@ def run_reference(args, wl):
     import oracle
     import synth
 
+    if wl["kind"] == "quantize":
+        # The oracle's block quantiser on 256-row samples of each shape.
+        g = np.random.default_rng(5)
+        samples = [g.standard_normal((256, K)).astype(np.float32) for (_, K, _) in wl["shapes"]]
+        per_step = max(0.02, 120.0 / (args.steps + args.warmup))
+        for _ in range(args.warmup):
+            oracle.quantize_blocks(samples[0], 1)
+        nbytes = secs = 0.0
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            while time.perf_counter() - t0 < per_step:
+                for xs in samples:
+                    oracle.quantize_blocks(xs, 1)
+                    nbytes += xs.size * 5
+            secs += time.perf_counter() - t0
+        value = nbytes / secs / 1e9
+        line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded N(0,1))", "config": {"workload": wl["desc"]}, "impl": "reference",
+                "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                 "sample": "256-row samples of each shape"},
+                "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
     # Inputs on the CPU (the reference arm uses no GPU); whole workload shapes.
     cases = []
     for c in build_cpu_cases(synth, wl):

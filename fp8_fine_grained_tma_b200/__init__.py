@@ -58,6 +58,7 @@ _SIG = {
     "fg_get_wait_limit_ns": (ctypes.c_ulonglong, []),
     "fg_query_block_n": (_I, [_I, _I, _I]),
     "fg_fp8_gemm_nt_small_m_no_alloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "fg_quantize_fp8_activations": (_I, [_P, _I, _P, _P, _I, _I, _P]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -167,6 +168,28 @@ def get_col_major_tma_aligned_tensor(sfa: torch.Tensor) -> torch.Tensor:
                "get_col_major_tma_aligned_tensor")
     out = storage.as_strided((G, M, KB), (KB * m_pad, 1, m_pad))
     return out[0] if squeeze else out
+
+
+def quantize_fp8_activations(x, stream=None):
+    """Row-wise 1x128 block quantisation of activations x [M, K] (float32 or
+    bfloat16, K % 128 == 0) into E4M3 codes and FP32 scales, the scales
+    already in the MN-major TMA-aligned layout: returns (q uint8 [M, K],
+    sfa view [M, K/128] with strides (1, M_pad)), ready for fp8_gemm_nt."""
+    if x.dtype not in (torch.float32, torch.bfloat16) or not x.is_cuda or x.dim() != 2:
+        raise TypeError("x must be a 2-D float32 or bfloat16 CUDA tensor")
+    x = x.contiguous()
+    M, K = x.shape
+    if K % BLOCK != 0:
+        raise ValueError("K must be a multiple of 128")
+    KB = K // BLOCK
+    m_pad = get_tma_aligned_size(M, 4)
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    storage = torch.empty(max(1, KB * m_pad), dtype=torch.float32, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(_lib.fg_quantize_fp8_activations(_ptr(x), 1 if x.dtype == torch.bfloat16 else 0, _ptr(q),
+                                                _ptr(storage), M, K, _stream(stream)),
+               "quantize_fp8_activations")
+    return q, storage[:KB * m_pad].as_strided((M, KB), (1, m_pad))
 
 
 def fp8_gemm_nt(A, sfa, B, sfb, D=None, stream=None):

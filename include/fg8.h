@@ -139,6 +139,22 @@ size_t fg_get_tma_aligned_size(size_t n, size_t elem_bytes);
  * Both pointers 16-byte aligned (in: 4).  Runs one small kernel on stream. */
 fg_status fg_transform_sfa_to_tma_layout(const float* in, float* out, int G, int M, int KB, fg_stream_t stream);
 
+/* Activation quantiser, the step that prepares A for the GEMMs (fine-grained
+ * scaling, chujupifa.com "机器之心报道", opening summary; the scale layout of
+ * get_col_major_tma_aligned_tensor, csdn page "实用工具").  For every 1 x 128
+ * block of a row of x:
+ *   scale = max(amax, 1e-4) / 448        in FP32 (448 = largest finite E4M3)
+ *   q     = E4M3(x / scale)              FP32 division, round to nearest even,
+ *                                        saturating at +-448
+ *   x   [M, K] FP32 (x_is_bf16 = 0) or BF16 (x_is_bf16 = 1), row-major
+ *   q   [M, K] E4M3 codes, row-major (written)
+ *   sfa [K/128][M_pad] FP32, MN-major, M_pad = fg_get_tma_aligned_size(M, 4)
+ *       (written, rows M .. M_pad-1 set to 0): the scale layout the GEMMs read.
+ * K must be a positive multiple of 128; x, q and sfa 16-byte aligned.  M == 0
+ * is a no-op.  Runs one kernel on stream. */
+fg_status fg_quantize_fp8_activations(const void* x, int x_is_bf16, void* q, float* sfa, int M, int K,
+                                      fg_stream_t stream);
+
 /* Reads and clears this device's status word after synchronising `stream`.
  * *code_out = 0 when no kernel recorded an error since the last call, else
  * FG_ERR_TIMEOUT; *detail_out (may be NULL) = (block << 8) | role of the

@@ -51,7 +51,7 @@ def test_binding_exposes_same_names():
                   "get_wait_limit_ns", "query_block_n", "get_num_sms", "set_num_sms",
                   "get_m_alignment_for_contiguous_layout", "get_tma_aligned_size",
                   "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
-                  "fp8_gemm_nt_small_m_no_alloc"):
+                  "fp8_gemm_nt_small_m_no_alloc", "quantize_fp8_activations"):
             assert hasattr(fg, py), py
     assert hasattr(fg, "get_col_major_tma_aligned_tensor")
 
@@ -117,6 +117,18 @@ def test_no_alloc_argument_checks(lib):
     assert f(FAKE + 8, FAKE, FAKE, FAKE, FAKE, 64, 128, 256, None) == FG_ERR_ALIGNMENT
     assert f(None, FAKE, FAKE, FAKE, FAKE, 64, 128, 256, None) == FG_ERR_INVALID_ARG
     assert f(None, None, None, None, None, 0, 128, 256, None) == FG_OK
+
+
+def test_quantiser_argument_checks(lib):
+    f = lib.fg_quantize_fp8_activations
+    f.argtypes = [P, ctypes.c_int, P, P, ctypes.c_int, ctypes.c_int, P]
+    f.restype = ctypes.c_int
+    assert f(FAKE, 0, FAKE, FAKE, 64, 200, None) == FG_ERR_UNSUPPORTED       # K % 128
+    assert f(FAKE, 2, FAKE, FAKE, 64, 256, None) == FG_ERR_INVALID_ARG       # dtype flag
+    assert f(FAKE, 0, FAKE, FAKE, -1, 256, None) == FG_ERR_INVALID_ARG
+    assert f(None, 0, FAKE, FAKE, 64, 256, None) == FG_ERR_INVALID_ARG
+    assert f(FAKE + 4, 0, FAKE, FAKE, 64, 256, None) == FG_ERR_ALIGNMENT
+    assert f(None, 0, None, None, 0, 256, None) == FG_OK                     # no rows: no-op
 
 
 def test_helpers(lib):
