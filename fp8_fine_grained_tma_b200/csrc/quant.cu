@@ -28,7 +28,7 @@ namespace fg8q {
 
 constexpr int QBLK = 128;
 constexpr int QTHREADS = 256;
-constexpr int QUNROLL = 4;   // blocks per warp whose loads are in flight together
+constexpr int QUNROLL = 2;   // blocks per warp whose loads are in flight together
 
 __device__ __forceinline__ float4 load4(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
 
@@ -51,7 +51,7 @@ __device__ __forceinline__ uint32_t to_e4m3x4(float a, float b, float c, float d
 }
 
 template <typename T>
-__global__ void __launch_bounds__(QTHREADS) quantize_kernel(const T* __restrict__ x, uint8_t* __restrict__ q,
+__global__ void __launch_bounds__(QTHREADS, 8) quantize_kernel(const T* __restrict__ x, uint8_t* __restrict__ q,
                                                             float* __restrict__ sfa, int M, int K, int m_pad) {
     const int KB = K / QBLK;
     const long long nblk = static_cast<long long>(M) * KB;
