@@ -389,11 +389,8 @@ def main(argv=None):
 
     flops_step = sum(c.flops for c in cases)
     bytes_step = sum(c.hbm_bytes for c in cases)
-    if pg is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    total_ms = max_over_ranks(total_ms, pg, device)
+    value = job_throughput(flops_step, world, args.steps, total_ms)
     unit = UNIT
     if flops_step == 0:   # a bandwidth-bound workload (the quantiser): GB/s
         value = world * sum(c.hbm_bytes for c in cases) * args.steps / (total_ms * 1e-3) / 1e9
@@ -523,14 +520,25 @@ def run_e2e(fg, cases, args, device, stream, pg, world):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if pg is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), pg, device)
     flops = sum(c.flops for c in cases) * steps * world
     return {"value": round(flops / (ms * 1e-3) / 1e12, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": round(ms / steps, 3)}
+
+
+def max_over_ranks(ms, pg, device):
+    """The slowest rank's time: every rank takes part, whatever its own value."""
+    if pg is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_rank_step, world, steps, total_ms):
+    """Whole-job TFLOPS: the work of all ranks (independent replicas, weak
+    scaling) over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (total_ms * 1e-3) / 1e12
 
 
 def read_traffic(workload):
