@@ -160,3 +160,20 @@ def test_block_n_choice_is_a_valid_width(lib):
         bn = abs(lib.fg_query_block_n(M, N, K))   # negative: the tile runs on a CTA pair
         assert 16 <= bn <= 256 and bn % 16 == 0
     assert lib.fg_query_block_n(64, 100, 128) == 0
+
+
+def test_c_program_links_and_checks_the_abi(lib, tmp_path):
+    """A plain C program, built with gcc against include/fg8.h and linked to
+    libfg8.so, runs the host-side checks without Python in between."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc") or shutil.which("cc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.join(ROOT, "fp8_fine_grained_tma_b200")
+    exe = str(tmp_path / "abi_check")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi", "abi_check.c"), "-L", libdir, "-lfg8",
+                    "-Wl,-rpath," + libdir, "-o", exe], check=True, capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
