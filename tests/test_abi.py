@@ -177,3 +177,26 @@ def test_c_program_links_and_checks_the_abi(lib, tmp_path):
                     "-Wl,-rpath," + libdir, "-o", exe], check=True, capture_output=True, text=True)
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stdout + r.stderr
+
+
+def test_binding_rejects_bad_tensors_before_any_launch():
+    """The Python binding validates dtypes, devices, shapes and layouts on the
+    host and raises before it reaches the library."""
+    import fp8_fine_grained_tma_b200 as fg
+    A = torch.zeros((64, 256), dtype=torch.uint8)          # CPU tensor
+    B = torch.zeros((128, 256), dtype=torch.uint8)
+    sfa = torch.zeros((64, 2), dtype=torch.float32)
+    sfb = torch.zeros((1, 2), dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA"):
+        fg.fp8_gemm_nt(A, sfa, B, sfb)
+    with pytest.raises(TypeError, match="E4M3"):
+        fg.fp8_gemm_nt(A.float(), sfa, B, sfb)
+    with pytest.raises(TypeError):
+        fg.quantize_fp8_activations(torch.zeros((4, 128), dtype=torch.float16))
+    with pytest.raises(TypeError):
+        fg.get_col_major_tma_aligned_tensor(torch.zeros((4, 2), dtype=torch.float64))
+    with pytest.raises(ValueError, match="divide 16"):
+        fg.get_tma_aligned_size(5, 3)
+    assert fg.get_tma_aligned_size(5, 4) == 8
+    assert fg.get_m_alignment_for_contiguous_layout() == 128
+    assert fg.status_string(6) == "FG_ERR_TIMEOUT"
