@@ -318,3 +318,30 @@ def test_compare_metric_properties():
     assert abs(c["diff"] - 2.0) < 1e-15
     c = oracle.compare(y * 1.01, y)
     assert 0 < c["diff"] < 1e-4
+
+
+# ------------------------------------------------------ randomised sweep --
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(M=st.integers(1, 40), nblk=st.integers(1, 3), N16=st.integers(1, 20), seed=st.integers(0, 2**31 - 1))
+def test_gemm_random_shapes_match_numpy(M, nblk, N16, seed):
+    """Random ragged shapes (M any, N any multiple of 16, K up to 3 blocks)
+    and random scales over many binades: the oracle equals the numpy float64
+    matmul of the dequantised operands."""
+    K, N = 128 * nblk, 16 * N16
+    A, sfa, B, sfb = rand_problem(M, N, K, seed)
+    assert_close(oracle.gemm_nt(A, sfa, B, sfb), dequant_ref(A, sfa, B, sfb))
+
+
+def test_synthetic_inputs_are_deterministic():
+    """The same seed gives the same bytes and scales (every parity test and
+    the bench rely on regenerating inputs on both sides)."""
+    a = synth.normal_inputs(33, 144, 256, seed=123)
+    b = synth.normal_inputs(33, 144, 256, seed=123)
+    c = synth.normal_inputs(33, 144, 256, seed=124)
+    for k in ("A", "sfa", "B", "sfb"):
+        assert torch.equal(getattr(a, k), getattr(b, k))
+    assert not torch.equal(a.A, c.A)
