@@ -57,6 +57,7 @@ _SIG = {
     "fg_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
     "fg_get_wait_limit_ns": (ctypes.c_ulonglong, []),
     "fg_query_block_n": (_I, [_I, _I, _I]),
+    "fg_query_plan": (_I, [_I, _I, _I, _I, _I, _I] + [ctypes.POINTER(_I)] * 5),
     "fg_fp8_gemm_nt_small_m_no_alloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "fg_quantize_fp8_activations": (_I, [_P, _I, _P, _P, _I, _I, _P]),
 }
@@ -315,3 +316,16 @@ def get_wait_limit_ns() -> int:
 
 def query_block_n(M: int, N: int, K: int) -> int:
     return _lib.fg_query_block_n(M, N, K)
+
+
+def query_plan(layout: str, rows: int, N: int, K: int, G: int = 1, expected_m: int = 0) -> dict:
+    """Launch plan of a GEMM call (diagnostics): which kernel, its tile width,
+    CTA pairs, K splits and cluster size.  layout: "normal", "contiguous" or
+    "masked"; rows = M, M_tot or M_max."""
+    lay = {"normal": 0, "contiguous": 1, "masked": 2}[layout]
+    out = [ctypes.c_int(0) for _ in range(5)]
+    _check(_lib.fg_query_plan(lay, int(rows), int(N), int(K), int(G), int(expected_m), *[ctypes.byref(o) for o in out]),
+           "query_plan")
+    kernel, tile_n, pair, splits, cluster = (o.value for o in out)
+    return {"kernel": "decode" if kernel == 1 else "tile", "tile_n": tile_n, "pair": bool(pair), "splits": splits,
+            "cluster": cluster}

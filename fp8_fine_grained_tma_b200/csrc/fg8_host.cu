@@ -739,6 +739,51 @@ int fg_query_block_n(int M, int N, int K) {
     return c.pair ? -c.bn : c.bn;
 }
 
+fg_status fg_query_plan(int layout, int rows, int N, int K, int G, int expected_m, int* kernel_out,
+                        int* tile_n_out, int* pair_out, int* splits_out, int* cluster_out) {
+    if (!kernel_out || !tile_n_out || !pair_out || !splits_out || !cluster_out) return FG_ERR_INVALID_ARG;
+    if (layout < LAYOUT_NORMAL || layout > LAYOUT_MASKED || rows <= 0 || N <= 0 || K <= 0 || G <= 0 ||
+        expected_m < 0)
+        return FG_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N % 16 != 0) return FG_ERR_UNSUPPORTED;
+    DeviceInfo* d = nullptr;
+    int sms = 148;
+    int dev_id = -1;
+    if (current_device(&d) == FG_OK) {
+        sms = effective_sms(*d);
+        cudaGetDevice(&dev_id);
+    } else if (g_num_sms.load() > 0) {
+        sms = g_num_sms.load();
+    }
+    if (layout == LAYOUT_NORMAL && rows <= std::min(decode_max_rows(), 256)) {
+        const int mt = decode_tile_width(rows);
+        const int stages = decode_stages(mt);
+        const size_t smem = decode_smem_bytes(BM * BK + mt * BK, stages, mt);
+        // Without a device the cluster residency cannot be queried: the plan
+        // then assumes no cluster launch (the workspace reduction).
+        const DecodePlan plan = dev_id >= 0 ? decode_plan(dev_id, mt, smem, stages * (BM * BK + mt * BK), N, K, sms)
+                                            : decode_plan(0, mt, smem, 0, N, K, sms);
+        *kernel_out = 1;
+        *tile_n_out = mt;
+        *pair_out = 0;
+        *splits_out = plan.splits;
+        *cluster_out = plan.cluster;
+        return FG_OK;
+    }
+    const int a_groups = layout == LAYOUT_MASKED ? G : 1;
+    const int hint = layout == LAYOUT_MASKED ? (expected_m > 0 ? std::min(expected_m, rows) : rows)
+                     : layout == LAYOUT_CONTIGUOUS ? BM : rows;
+    const double hbm = static_cast<double>(a_groups) * std::min(rows, std::max(1, hint)) * K +
+                       static_cast<double>(G) * N * K + 2.0 * a_groups * rows * N;
+    const Choice c = choose_config(layout, rows, a_groups, layout == LAYOUT_MASKED ? hint : rows, N, K, sms, hbm);
+    *kernel_out = 0;
+    *tile_n_out = c.bn;
+    *pair_out = c.pair ? 1 : 0;
+    *splits_out = 1;
+    *cluster_out = c.pair ? 2 : 1;
+    return FG_OK;
+}
+
 }  // extern "C"
 
 // ---- few-rows GEMM on library-owned scratch (fg_fp8_gemm_nt_small_m_no_alloc) --

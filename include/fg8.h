@@ -174,6 +174,23 @@ unsigned long long fg_get_wait_limit_ns(void);
  * tiles), or 0 for an unsupported shape.  Diagnostics. */
 int fg_query_block_n(int M, int N, int K);
 
+/* The launch plan a GEMM call of these sizes would use with the current SM
+ * budget and environment (diagnostics; launches nothing, allocates nothing).
+ *   layout 0 = normal (rows = M, G = 1), 1 = contiguous (rows = M_tot, G
+ *   experts), 2 = masked (rows = M_max, G groups, expected_m as in the call).
+ * Outputs (all required):
+ *   *kernel_out  0 = the persistent tile kernel, 1 = the few-rows (decode) kernel
+ *   *tile_n_out  BLOCK_N of the tile kernel, or the token-tile width of the
+ *                decode kernel
+ *   *pair_out    1 when tiles run on CTA pairs (256-row tiles)
+ *   *splits_out  K splits per output tile (decode kernel; 1 otherwise)
+ *   *cluster_out CTAs per cluster (split-K reduction through distributed
+ *                shared memory when equal to *splits_out > 1)
+ * Returns FG_ERR_INVALID_ARG for a bad layout, non-positive sizes or a NULL
+ * output, FG_ERR_UNSUPPORTED when K % 128 != 0 or N % 16 != 0. */
+fg_status fg_query_plan(int layout, int rows, int N, int K, int G, int expected_m, int* kernel_out,
+                        int* tile_n_out, int* pair_out, int* splits_out, int* cluster_out);
+
 /*
  * Few-rows normal GEMM that allocates nothing.  The pages have no counterpart
  * to this entry point: it is an addition of this library.

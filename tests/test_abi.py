@@ -51,7 +51,7 @@ def test_binding_exposes_same_names():
                   "get_wait_limit_ns", "query_block_n", "get_num_sms", "set_num_sms",
                   "get_m_alignment_for_contiguous_layout", "get_tma_aligned_size",
                   "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
-                  "fp8_gemm_nt_small_m_no_alloc", "quantize_fp8_activations"):
+                  "fp8_gemm_nt_small_m_no_alloc", "quantize_fp8_activations", "query_plan"):
             assert hasattr(fg, py), py
     assert hasattr(fg, "get_col_major_tma_aligned_tensor")
 
@@ -160,6 +160,24 @@ def test_block_n_choice_is_a_valid_width(lib):
         bn = abs(lib.fg_query_block_n(M, N, K))   # negative: the tile runs on a CTA pair
         assert 16 <= bn <= 256 and bn % 16 == 0
     assert lib.fg_query_block_n(64, 100, 128) == 0
+
+
+def test_plan_query_without_a_device():
+    """The plan query is host logic: small M goes to the few-rows kernel with
+    a token-tile width covering M, larger M to the tile kernel with a block
+    width in 16..256; bad arguments are rejected."""
+    import fp8_fine_grained_tma_b200 as fg
+    p = fg.query_plan("normal", 64, 2112, 7168)
+    assert p["kernel"] == "decode" and p["tile_n"] == 64 and 1 <= p["splits"] <= 56
+    p = fg.query_plan("normal", 100, 4096, 7168)
+    assert p["kernel"] == "decode" and p["tile_n"] == 128
+    for layout, rows, G, em in [("normal", 4096, 1, 0), ("contiguous", 37376, 8, 0), ("masked", 256, 32, 128)]:
+        p = fg.query_plan(layout, rows, 7168, 2048, G, em)
+        assert p["kernel"] == "tile" and 16 <= p["tile_n"] <= 256 and p["tile_n"] % 16 == 0 and p["splits"] == 1
+    with pytest.raises(fg.FG8Error):
+        fg.query_plan("normal", 64, 2112, 100)
+    with pytest.raises(fg.FG8Error):
+        fg.query_plan("normal", 0, 2112, 128)
 
 
 def test_c_program_links_and_checks_the_abi(lib, tmp_path):

@@ -269,6 +269,41 @@ def sample_rows(M, n, seed):
     return np.array(sorted(rows))
 
 
+def block_edge_rows(M, n, seed):
+    """The first and last row of every 128-row block (so every row tile of the
+    kernel is checked on both sides of its boundaries) plus n random rows."""
+    rows = set(sample_rows(M, n, seed).tolist())
+    for b0 in range(0, M, 128):
+        rows.add(b0)
+        rows.add(min(M, b0 + 128) - 1)
+    return np.array(sorted(rows))
+
+
+def stratified_written_rows(written, labels, seed, per_segment=2):
+    """Rows to check in a grouped output whose written rows form segments
+    (runs of consecutive written rows with the same label: expert or group):
+    the first and last written row of every segment, the written rows on
+    either side of every 128-row block boundary inside it, and per_segment
+    random rows of it."""
+    rng = np.random.default_rng(seed)
+    idx = np.nonzero(written)[0]
+    if len(idx) == 0:
+        return idx
+    lab = np.asarray(labels)[idx]
+    brk = (np.diff(idx) != 1) | (np.diff(lab) != 0)
+    starts = np.concatenate([[0], np.nonzero(brk)[0] + 1])
+    ends = np.concatenate([starts[1:], [len(idx)]])
+    rows = set()
+    for a, b in zip(starts, ends):
+        seg = idx[a:b]
+        rows |= {int(seg[0]), int(seg[-1])}
+        rows |= set(int(r) for r in rng.choice(seg, min(per_segment, len(seg)), replace=False))
+        for r in seg:
+            if r % 128 == 0 or r % 128 == 127:
+                rows.add(int(r))
+    return np.array(sorted(rows))
+
+
 def test_decode_config_full(fg):
     x = synth.normal_inputs(64, 2112, 7168, seed=synth.seed_for(0, 0))
     A, sfa, B, sfb = to_gpu_normal(fg, x)
@@ -285,26 +320,53 @@ def test_prefill_config_sampled_rows(fg, si, N, K):
     A, sfa, B, sfb = to_gpu_normal(fg, x)
     D = fg.fp8_gemm_nt(A, sfa, B, sfb)
     torch.cuda.synchronize()
-    rows = sample_rows(M, 24, si)
+    rows = block_edge_rows(M, 24, si)
     ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), rows=rows)
     check(D[torch.from_numpy(rows).cuda()].double().cpu().numpy(), ref)
 
 
 @pytest.mark.parametrize("si,N,K", [(0, 4096, 7168), (1, 7168, 2048)])
 def test_contiguous_config_sampled_rows(fg, si, N, K):
+    """Every expert is value-checked (first and last row, rows at each
+    128-row block boundary, random rows), each against its own B and sfb."""
     x = synth.contiguous_inputs(8, N, K, seed=synth.seed_for(2, si))
     D = run_contiguous(fg, x)
-    real = np.nonzero(x.m_indices.numpy() >= 0)[0]
-    rng = np.random.default_rng(si)
-    rows = np.sort(rng.choice(real, 32, replace=False))
-    check_contiguous(fg, x, D, rows=rows)
+    mi = x.m_indices.numpy()
+    rows = stratified_written_rows(mi >= 0, mi, si)
+    assert set(mi[rows].tolist()) == {e for e in range(8) if x.counts[e] > 0}
+    Dc = D.cpu()
+    assert torch.all(Dc[torch.from_numpy(mi < 0)].view(torch.int16) == sentinel_bf16().view(torch.int16))
+    ref, written = oracle.m_grouped_contiguous(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), mi,
+                                               rows=rows)
+    assert written.all()
+    got = Dc[torch.from_numpy(rows)].double().numpy()
+    check(got, ref)
+    for e in range(8):   # each expert's rows also meet the tolerance on their own
+        sel = mi[rows] == e
+        if sel.any():
+            check(got[sel], ref[sel])
 
 
 @pytest.mark.parametrize("si,N,K", [(0, 4096, 7168), (1, 7168, 2048)])
 def test_masked_config_sampled_rows(fg, si, N, K):
+    """Every non-empty group is value-checked (first and last row, rows at the
+    128-row boundary, random rows), each against its own B and sfb."""
     x = synth.masked_inputs(32, 256, N, K, seed=synth.seed_for(3, si))
     D = run_masked(fg, x, expected_m=128)
-    check_masked(fg, x, D, sample=32)
+    check_masked(fg, x, D, sample=0)
+    mm = x.masked_m.numpy()
+    lim = np.minimum(np.maximum(mm, 0), x.M_max)
+    written = (np.arange(x.M_max)[None, :] < lim[:, None]).reshape(-1)
+    rows = stratified_written_rows(written, np.arange(len(written)) // x.M_max, si)
+    assert set((rows // x.M_max).tolist()) == {g for g in range(x.G) if lim[g] > 0}
+    flat = D.view(-1, x.N)
+    ref, w = oracle.m_grouped_masked(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), mm, rows=rows)
+    assert w.all()
+    check(flat[torch.from_numpy(rows).cuda()].double().cpu().numpy(), ref)
+    for g in range(x.G):   # each group also meets the tolerance on its own
+        sel = (rows // x.M_max) == g
+        if sel.any():
+            check(flat[torch.from_numpy(rows[sel]).cuda()].double().cpu().numpy(), ref[sel])
 
 
 @pytest.mark.parametrize("si,M,N,K", [(i * 2 + j, M, N, K) for j, M in enumerate([64, 128])

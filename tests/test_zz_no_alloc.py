@@ -5,10 +5,10 @@ while they run: a serving engine that reserved nearly all device memory for
 its own pool up front, or a latency-critical loop where an allocation (which
 may synchronise the device) is not allowed.  It keeps its split-K partial sums
 and counters in a device array that the library itself holds, so this test
-checks, through the C ABI, that it gives what fg_fp8_gemm_nt gives (within the
-parity tolerance of the other GPU tests) on calls made back to back, each
-reusing the scratch that the previous one left behind, and that those calls
-leave the device's free memory unchanged.
+checks, through the C ABI, that its results match the CPU oracle and what
+fg_fp8_gemm_nt gives (within the parity tolerance of the other GPU tests) on
+calls made back to back, each reusing the scratch that the previous one left
+behind, and that those calls leave the device's free memory unchanged.
 
 The file is named so that pytest collects it last.
 """
@@ -17,6 +17,8 @@ import ctypes
 import numpy as np
 import pytest
 import torch
+
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -46,12 +48,14 @@ def lib(fg):
 
 
 def inputs(fg, M, N, K, seed):
-    """E4M3 operands with per-block scales, made on the device."""
+    """E4M3 operands with per-block scales (made on the host, uploaded), and
+    the CPU oracle's FP64 result for them."""
     import synth
     x = synth.normal_inputs(M, N, K, seed=seed)
     A, B, sfb = x.A.cuda(), x.B.cuda(), x.sfb.cuda()
     sfa = fg.get_col_major_tma_aligned_tensor(x.sfa.cuda())
-    return A, sfa, B, sfb
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    return (A, sfa, B, sfb), ref
 
 
 def call(fn, ops, D):
@@ -62,9 +66,11 @@ def call(fn, ops, D):
     return fn(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(), D.data_ptr(), M, N, K, stream)
 
 
-def close(x: torch.Tensor, y: torch.Tensor):
+def close(x: torch.Tensor, y):
+    """Parity metric of the GPU tests: x (bf16 result) against y (the oracle's
+    FP64 result, or another bf16 result)."""
     x = x.double().cpu().numpy()
-    y = y.double().cpu().numpy()
+    y = y.double().cpu().numpy() if isinstance(y, torch.Tensor) else np.asarray(y, dtype=np.float64)
     assert np.all(np.isfinite(x))
     diff = 1.0 - 2.0 * np.sum(x * y) / max(np.sum(x * x + y * y), 1e-300)
     assert diff <= DIFF_TOL, diff
@@ -81,8 +87,8 @@ CASES = [(64, 2112, 7168, None), (17, 768, 2048, "5"), (200, 1024, 4096, "6"), (
 def test_no_alloc_matches_the_normal_entry_point(fg, lib, M, N, K, splits, monkeypatch):
     if splits:
         monkeypatch.setenv("FG_FORCE_SPLITS", splits)
-    ops = inputs(fg, M, N, K, seed=20261000 + M)
-    other = inputs(fg, 40, 528, 3072, seed=20261999)   # a second shape between the two calls
+    ops, oracle_ref = inputs(fg, M, N, K, seed=20261000 + M)
+    other, oracle_other = inputs(fg, 40, 528, 3072, seed=20261999)   # a second shape between the two calls
     ref = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     assert call(lib.fg_fp8_gemm_nt, ops, ref) == 0
     ref_other = torch.empty((40, 528), dtype=torch.bfloat16, device="cuda")
@@ -107,16 +113,19 @@ def test_no_alloc_matches_the_normal_entry_point(fg, lib, M, N, K, splits, monke
 
     code, detail = fg.get_last_device_status()
     assert code == 0, (code, detail)
+    # Each result against the CPU oracle (FP64), and against the normal entry point.
+    close(outs[0], oracle_ref)
+    close(outs[1], oracle_ref)
+    close(out_other, oracle_other)
     close(outs[0], ref)
-    close(outs[1], ref)
     close(out_other, ref_other)
     assert torch.equal(outs[0], outs[1])   # the later call ran on the scratch the others left behind
     assert free_after == free_before
 
 
 def test_no_alloc_rejects_sizes_beyond_its_limits(fg, lib):
-    ops = inputs(fg, 64, 256, 256, seed=20261998)
-    big_m = inputs(fg, 257, 256, 256, seed=20261997)
+    ops, _ = inputs(fg, 64, 256, 256, seed=20261998)
+    big_m, _ = inputs(fg, 257, 256, 256, seed=20261997)
     D = torch.empty((257, 256), dtype=torch.bfloat16, device="cuda")
     assert call(lib.fg_fp8_gemm_nt_small_m_no_alloc, big_m, D) == FG_ERR_UNSUPPORTED
     A, sfa, B, sfb = ops
