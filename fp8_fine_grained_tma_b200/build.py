@@ -27,7 +27,8 @@ LIB = os.path.join(PKG, "libfg8.so")
 BLOCK_NS = list(range(16, 257, 16))
 DECODE_MTS = list(range(32, 257, 32))
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
+FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE,
+         "-I", CSRC]
 
 
 def nvcc() -> str:

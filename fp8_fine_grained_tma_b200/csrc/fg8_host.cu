@@ -155,37 +155,77 @@ fg_status operand_map(const void* ptr, uint64_t K, uint64_t rows, uint64_t group
     return FG_OK;
 }
 
+// 3-D BF16 output D [groups][rows][N] (N innermost), box 16 (N) x 32 rows x 1,
+// 32-byte swizzle: the pieces the GEMM kernel's epilogue stores by TMA.  The
+// map's extents clip the stores at N columns and `rows` rows.
+struct OutKey {
+    const void* ptr;
+    uint64_t N, rows, groups;
+    bool operator<(const OutKey& o) const {
+        return std::tie(ptr, N, rows, groups) < std::tie(o.ptr, o.N, o.rows, o.groups);
+    }
+};
+std::map<OutKey, CUtensorMap> g_out_maps;
+
+fg_status output_map(void* ptr, uint64_t N, uint64_t rows, uint64_t groups, CUtensorMap* out) {
+    OutKey key{ptr, N, rows, groups};
+    {
+        std::lock_guard<std::mutex> lk(g_maps_mutex);
+        auto it = g_out_maps.find(key);
+        if (it != g_out_maps.end()) {
+            *out = it->second;
+            return FG_OK;
+        }
+    }
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return FG_ERR_NO_DEVICE;
+    CUtensorMap m;
+    std::memset(&m, 0, sizeof(m));
+    const cuuint64_t dims[3] = {N, rows, groups};
+    const cuuint64_t strides[2] = {N * 2, N * 2 * rows};   // bytes, dims 1 and 2
+    const cuuint32_t box[3] = {16, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return FG_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lk(g_maps_mutex);
+        if (g_out_maps.size() > 512) g_out_maps.clear();
+        g_out_maps[key] = m;
+    }
+    *out = m;
+    return FG_OK;
+}
+
 // ---- configuration -----------------------------------------------------------
 // Cost model of one candidate (block width BN, 128-row tiles on one CTA or
-// 256-row tiles on a CTA pair), in SM clock cycles.  Per K block a tile needs
-//   max(MMA, promotion cycle, operand loads) cycles:
-//   MMA = 2*BN (8192 E4M3 MAC/clk/SM: each SM computes 128 x BN x 128),
-//   promotion cycle = 240 + 5*BN (measured on B200: the promotion warps' read /
-//           scale / accumulate / release cycle per K block, which the two to
-//           four TMEM accumulators cannot fully hide),
-//   loads = (A rows loaded * 128 + 128*BNL) / 44 B/clk (the L2 -> SM rate the
-//           kernel reaches when the tensor cores are idle),
-// with BNL = BN rows of B per CTA (BN/2 on a pair).  Tiles per CTA (pair) =
-// ceil(tiles / (SMs or SMs/2)); each tile adds an epilogue of ~2*BN + 800.
-// The job is bounded below by its unique HBM bytes at ~3.5 KB/clk.
+// 256-row tiles on a CTA pair), in SM clock cycles, from measurements on B200:
+//   - the tensor core needs ~512 cycles per K block of a 128-row tile for any
+//     BN <= 256 (one M=128, K=32 MMA every ~128 cycles), so wider blocks do
+//     more work in the same time;
+//   - with two TMEM accumulators (BN > 170) the promotion of one K block and
+//     its handshake with the MMA issuers stretch that to ~700 cycles; three
+//     (BN <= 170) to ~600; four (BN <= 128) to ~520;
+//   - each tile adds an epilogue of ~2000 cycles that overlaps the next tile
+//     only partly.
+// Tiles per CTA (pair) = ceil(tiles / (SMs or SMs/2)).  The job is bounded
+// below by its unique HBM bytes at ~3.3 KB/clk.
 struct Choice {
     int bn = 0;
     bool pair = false;
 };
 
-double estimate_cycles(bool pair, int bn, long long row_tiles, int a_rows, int N, int K, int num_sms,
-                       double hbm_bytes) {
+double estimate_cycles(bool pair, int bn, long long row_tiles, int N, int K, int num_sms, double hbm_bytes) {
     const int KB = K / BK;
-    const int bnl = pair ? bn / 2 : bn;
     const long long tiles = row_tiles * ((N + bn - 1) / bn);
     const int units = std::max(1, pair ? num_sms / 2 : num_sms);
     const double waves = static_cast<double>((tiles + units - 1) / units);
-    const double mma = 2.0 * bn;
-    const double promotion = 240.0 + 5.0 * bn;
-    const double loads = (a_rows * 128.0 + 128.0 * bnl) / 44.0;
-    const double per_kb = std::max(mma, std::max(promotion, loads));
-    const double t_tiles = waves * (KB * per_kb + 2.0 * bn + 800.0);
-    return std::max(t_tiles, hbm_bytes / 3500.0) + 2000.0;
+    const int acc_stride = (bn + 31) / 32 * 32;
+    const int nbuf = std::min(4, 512 / acc_stride);
+    const double per_kb = nbuf >= 4 ? 520.0 : (nbuf == 3 ? 600.0 : 700.0);
+    const double t_tiles = waves * (KB * per_kb + 2000.0);
+    return std::max(t_tiles, hbm_bytes / 3300.0) + 2000.0;
 }
 
 // rows: rows per row group; groups: row groups (masked: G, else 1); valid_rows:
@@ -208,8 +248,7 @@ Choice choose_config(int layout, int rows, int groups, int valid_rows, int N, in
             if (fbn >= 16 && fbn <= 256 && fbn % 16 == 0 && bn != fbn) continue;
             const int tile_m = pair ? 2 * BM : BM;
             const long long row_tiles = static_cast<long long>(groups) * ((valid_rows + tile_m - 1) / tile_m);
-            const int a_rows = std::min(BM, std::max(1, valid_rows));
-            const double t = estimate_cycles(pair, bn, std::max(1ll, row_tiles), a_rows, N, K, num_sms, hbm_bytes);
+            const double t = estimate_cycles(pair, bn, std::max(1ll, row_tiles), N, K, num_sms, hbm_bytes);
             if (t < best_t * 0.999 || (t <= best_t * 1.001 && (pair > (best.pair ? 1 : 0) || bn > best.bn))) {
                 if (t < best_t) best_t = t;
                 best.bn = bn;
@@ -227,28 +266,28 @@ int stage_bytes_for(int bn, bool pair) { return BM * BK + (pair ? bn / 2 : bn) *
 int choose_stages(int bn, bool pair) {
     const int sb = stage_bytes_for(bn, pair);
     int s = 8;
-    while (s > MAX_NBUF && gemm_smem_bytes(sb, s) > static_cast<size_t>(kMaxDynamicSmem)) --s;
+    while (s > MAX_NBUF && gemm_smem_bytes(sb, s, pair) > static_cast<size_t>(kMaxDynamicSmem)) --s;
     return s;
 }
 
 template <int BN>
-cudaError_t launch_either(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
-                          size_t smem, cudaStream_t st) {
+cudaError_t launch_either(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                          const GemmParams& p, int grid, size_t smem, cudaStream_t st) {
     if constexpr (BN >= 32) {
-        if (pair) return launch_gemm<BN, true>(ta, tb, p, grid, smem, st);
+        if (pair) return launch_gemm<BN, true>(ta, tb, td, p, grid, smem, st);
     } else {
         if (pair) return cudaErrorInvalidValue;
     }
-    return launch_gemm<BN, false>(ta, tb, p, grid, smem, st);
+    return launch_gemm<BN, false>(ta, tb, td, p, grid, smem, st);
 }
 
-fg_status launch_bn(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
-                    size_t smem, cudaStream_t st) {
+fg_status launch_bn(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                    const GemmParams& p, int grid, size_t smem, cudaStream_t st) {
     cudaError_t e = cudaErrorInvalidValue;
     switch (bn) {
 #define FG8_CASE(BNV) \
     case BNV:         \
-        e = launch_either<BNV>(pair, ta, tb, p, grid, smem, st); \
+        e = launch_either<BNV>(pair, ta, tb, td, p, grid, smem, st); \
         break;
         FG8_FOR_EACH_BN(FG8_CASE)
 #undef FG8_CASE
@@ -514,12 +553,14 @@ fg_status run_gemm(int layout, const void* A, const float* sfa, const void* B, c
     const int bn = c.bn;
     const int tile_m = c.pair ? 2 * BM : BM;
     const int stages = choose_stages(bn, c.pair);
-    const size_t smem = gemm_smem_bytes(stage_bytes_for(bn, c.pair), stages);
+    const size_t smem = gemm_smem_bytes(stage_bytes_for(bn, c.pair), stages, c.pair);
 
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, td;
     st = operand_map(A, K, rows, a_groups, BM, &ta);
     if (st != FG_OK) return st;
     st = operand_map(B, K, N, G, c.pair ? bn / 2 : bn, &tb);
+    if (st != FG_OK) return st;
+    st = output_map(D, N, rows, a_groups, &td);
     if (st != FG_OK) return st;
 
     GemmParams p;
@@ -551,7 +592,7 @@ fg_status run_gemm(int layout, const void* A, const float* sfa, const void* B, c
     const int units = c.pair ? num_sms / 2 : num_sms;
     const long long used = std::max<long long>(1, std::min<long long>(tiles, units));
     const int grid = static_cast<int>(c.pair ? 2 * used : used);
-    return launch_bn(bn, c.pair, ta, tb, p, grid, smem, stream);
+    return launch_bn(bn, c.pair, ta, tb, td, p, grid, smem, stream);
 }
 
 __global__ void sfa_transform_kernel(const float* __restrict__ in, float* __restrict__ out, int G, int M, int KB,

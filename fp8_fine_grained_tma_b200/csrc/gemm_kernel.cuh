@@ -19,16 +19,20 @@
 //   warps 0-7  promotion + epilogue: two warpgroups split the tile's 16-column
 //              chunks; each thread owns one TMEM lane (= one output row), reads
 //              the block's partial sums with tcgen05.ld, multiplies by
-//              sfa[m,kb] * sfb[n/128,kb] and adds into FP32 registers; after
-//              the last block it converts to BF16 and stores the rows that may
-//              be written.
+//              sfa[m,kb] * sfb[n/128,kb] (loaded by the thread itself a group of
+//              K blocks ahead) and adds into FP32 registers; after the last
+//              block it converts to BF16 and stores its 32 x 16 pieces with TMA
+//              bulk tensor stores (rows that may not be written go through
+//              predicated stores instead).
 //   warp 11    idle (it completes the third warpgroup for the register split).
+// The tensor core takes about the same time per K block for any N up to 256
+// (one 128-row MMA of K=32 every ~128 cycles), so the widest block (256)
+// gives the most work per K block; narrower blocks exist for small N.
 // PAIR = false: the tile is 128 x BN and the CTA works alone (M=128 MMA).
 // PAIR = true:  two CTAs of a cluster share a 256 x BN tile (tcgen05
 //   cta_group::2, M=256): each loads its own 128 rows of A and its own half of
 //   the BN rows of B, the leader CTA issues the MMAs, and each CTA's TMEM holds
-//   its 128 rows x BN columns.  Each SM then moves 16 KiB + BN/2 * 128 bytes per
-//   K block instead of 16 KiB + BN * 128.  No load uses multicast.
+//   its 128 rows x BN columns.  No load uses multicast.
 // Tiles are scheduled persistently (static stride over a raster-grouped tile
 // order); the contiguous and masked MoE layouts of the pages (game.3loumao.org
 // explainer, section "03 DeepSeek是如何创新的？") change only the tile -> (group,
@@ -59,9 +63,15 @@ constexpr int REGS_LAUNCH = 168;
 constexpr int REGS_PRODUCER = 56;
 constexpr int REGS_PROMOTION = 224;
 static_assert(256 * REGS_PROMOTION + 128 * REGS_PRODUCER <= NUM_THREADS * REGS_LAUNCH, "register split");
-constexpr int EPI_COLS = 32;                       // columns per staged piece
-constexpr int EPI_PITCH = EPI_COLS * 2 + 16;       // bytes per staged row (padding kills bank conflicts)
-constexpr int EPI_WARP_BYTES = 32 * EPI_PITCH;     // staging bytes per epilogue warp
+// Epilogue staging: per promotion warp EPI_SLOTS pieces of 32 rows x 16 BF16
+// columns (32 bytes a row, in the 32-byte swizzle of the D tensor map: the
+// 16-byte half h of row r sits at r*32 + (h ^ ((r >> 2) & 1)) * 16).
+constexpr int EPI_SLOT_BYTES = 32 * 32;
+constexpr int EPI_SLOTS = 2;
+constexpr int EPI_WARP_BYTES = EPI_SLOTS * EPI_SLOT_BYTES;
+// Scales are loaded by the promotion threads themselves, SCALE_GROUP K blocks
+// at a time, one group ahead of their use.
+constexpr int SCALE_GROUP = 2;
 constexpr int A_TILE_BYTES = BM * BK;              // 16 KiB
 // Contiguous layout, CTA pairs: the 128-row blocks that start a pair tile are
 // listed in shared memory (one 16-bit block index each).
@@ -125,11 +135,12 @@ struct GemmShape {
 };
 
 // Dynamic shared memory layout (after aligning the base to 1024 bytes):
-//   [stages x (A tile | B tile)] [8 x epilogue staging] [pair list] [barriers] [tmem slot, abort flag, list count]
+//   [stages x (A tile | B tile)] [8 x epilogue staging] [pair list (pairs only)]
+//   [barriers] [tmem slot, abort flag, list count]
 constexpr int MAX_NBUF = 4;
-__host__ __device__ constexpr size_t gemm_smem_bytes(int stage_bytes, int stages) {
-    return 1024 + static_cast<size_t>(stages) * stage_bytes + NUM_EPI_WARPS * EPI_WARP_BYTES + PAIR_LIST_BYTES +
-           (2 * stages + 2 * MAX_NBUF + 1) * 8 + 16;
+__host__ __device__ constexpr size_t gemm_smem_bytes(int stage_bytes, int stages, bool pair) {
+    return 1024 + static_cast<size_t>(stages) * stage_bytes + NUM_EPI_WARPS * EPI_WARP_BYTES +
+           (pair ? PAIR_LIST_BYTES : 0) + (2 * stages + 2 * MAX_NBUF + 1) * 8 + 16;
 }
 
 struct TileInfo {
@@ -277,14 +288,25 @@ __device__ __forceinline__ int build_pair_list(const GemmParams& p, int* tags, u
     return count < MAX_PAIR_LIST ? count : MAX_PAIR_LIST;
 }
 
+// BF16 pair of (lo, hi), round to nearest even, as one 32-bit word.
+__device__ __forceinline__ uint4 pack_bf16x8(const float2 (&a)[8], int q) {
+    uint4 v;
+    v.x = pack_bf16x2(a[4 * q + 0].x, a[4 * q + 0].y);
+    v.y = pack_bf16x2(a[4 * q + 1].x, a[4 * q + 1].y);
+    v.z = pack_bf16x2(a[4 * q + 2].x, a[4 * q + 2].y);
+    v.w = pack_bf16x2(a[4 * q + 3].x, a[4 * q + 3].y);
+    return v;
+}
+
 template <int BN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fg8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
     using S = GemmShape<BN, PAIR>;
     constexpr int NC = S::NC;
     constexpr int CPW = S::CPW;
-    constexpr int LB = CPW <= 4 ? CPW : 4;   // chunks read from TMEM per wait
+    constexpr int PB = CPW <= 2 ? CPW : 2;   // chunks per TMEM load batch of the promotion pipeline
+    constexpr int NBATCH = (CPW + PB - 1) / PB;
     constexpr uint32_t IDESC = ptx::idesc_e4m3_f32(S::TILE_M, BN);
 
     extern __shared__ uint8_t smem_raw[];
@@ -292,7 +314,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t* stage_base = smem;
     uint8_t* epi_base = smem + static_cast<size_t>(p.stages) * S::STAGE_BYTES;
     uint16_t* pair_list = reinterpret_cast<uint16_t*>(epi_base + NUM_EPI_WARPS * EPI_WARP_BYTES);
-    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(pair_list) + PAIR_LIST_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(pair_list) + (PAIR ? PAIR_LIST_BYTES : 0));
     uint64_t* empty = full + p.stages;
     uint64_t* tfull = empty + p.stages;
     uint64_t* tempty = tfull + S::NBUF;
@@ -324,6 +346,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::fence_mbarrier_init();
         ptx::prefetch_tensormap(&tmA);
         ptx::prefetch_tensormap(&tmB);
+        ptx::prefetch_tensormap(&tmD);
     }
     if (warp == MMA_WARP) {
         if constexpr (PAIR) {
@@ -476,6 +499,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         const int chunk0 = wg * CPW;                  // first 16-column chunk of this warpgroup
         uint8_t* stg = epi_base + warp * EPI_WARP_BYTES;
+        const uint32_t tempty_peer0 = PAIR ? ptx::mapa_shared(ptx::smem_addr(&tempty[0]), 0) : 0u;
 
         TileScheduler<PAIR> sch(unit, num_units, rank, pair_list, pair_count);
         TileInfo t;
@@ -484,15 +508,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bool ok = true;
         while (ok && sch.get(p, t)) {
             const int row = t.row0 + row_in_tile;
-            const bool row_in = row < p.rows;
-            const int a_g = p.layout == LAYOUT_MASKED ? t.g : 0;
-            const float* sfa_p = p.sfa + static_cast<size_t>(a_g) * p.KB * p.sfa_ld + row;
-            const float* sfb_p = p.sfb + static_cast<size_t>(t.g) * p.NB * p.KB;
             const int n0 = t.n_blk * BN;
-            const int my_n0 = n0 + chunk0 * 16;
-            const int nb_lo = min(my_n0 / 128, p.NB - 1);
+            // Scale block of this warpgroup's chunks: nb_lo for the first chunk,
+            // nb_hi for the chunks whose bit is set in hi_mask (a warpgroup spans
+            // <= 128 columns, so at most two blocks).  Block widths that are
+            // multiples of 128 start every tile on a block boundary, so a
+            // warpgroup then lies in a single block.  Blocks past the last one
+            // (columns >= N, never stored) are clamped to it.
+            const int nb_lo = min((n0 + chunk0 * 16) / 128, p.NB - 1);
             const int nb_hi = min(nb_lo + 1, p.NB - 1);
-            const int split_col = (my_n0 / 128 + 1) * 128;   // chunk columns at or past this use nb_hi
+            uint32_t hi_mask = 0;
+            if constexpr (BN % 128 != 0) {
+#pragma unroll
+                for (int i = 0; i < CPW; ++i)
+                    if ((n0 + (chunk0 + i) * 16) / 128 > (n0 + chunk0 * 16) / 128) hi_mask |= 1u << i;
+            }
+            // This row's sfa (rows past the padded scale array read nothing:
+            // they are never stored) and the warpgroup's sfb rows.
+            const int a_g = p.layout == LAYOUT_MASKED ? t.g : 0;
+            const bool row_has_scale = row < p.sfa_ld;
+            const float* sfa_row = p.sfa + static_cast<size_t>(a_g) * p.KB * p.sfa_ld + (row_has_scale ? row : 0);
+            const float* sfb_lo = p.sfb + (static_cast<size_t>(t.g) * p.NB + nb_lo) * p.KB;
+            const float* sfb_hi = p.sfb + (static_cast<size_t>(t.g) * p.NB + nb_hi) * p.KB;
 
             // Column pairs: the promotion uses the packed FP32 FMA (two FMAs per
             // instruction, each rounded to nearest as a scalar fmaf would be).
@@ -502,149 +539,185 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
 
-            // Scales are fetched SCALE_AHEAD K blocks ahead into a small register
-            // ring, so a block's scale products never wait on a global load.
-            constexpr int SCALE_AHEAD = 3;
-            const float* sfb_lo = sfb_p + static_cast<size_t>(nb_lo) * p.KB;
-            const float* sfb_hi = sfb_p + static_cast<size_t>(nb_hi) * p.KB;
-            float ra[SCALE_AHEAD], rl[SCALE_AHEAD], rh[SCALE_AHEAD];
+            // Scales: the raw values of the next group of SCALE_GROUP K blocks are
+            // loaded while the current group is promoted (their latency is
+            // hidden behind a group's MMAs); at the group switch they become
+            // the per-K-block factors sfa * sfb of the current group.  With two
+            // accumulators the promotion's latency bounds the tensor core's
+            // rate, so no load or shared-memory access of scales sits between
+            // an accumulator's completion and its release.
+            float na[SCALE_GROUP], nl[SCALE_GROUP], nh[SCALE_GROUP];
+#define FG8_LOAD_SCALE_GROUP(KG)                                                                      \
+    _Pragma("unroll") for (int u = 0; u < SCALE_GROUP; ++u) {                                         \
+        const int kq = min((KG) + u, p.KB - 1);                                                       \
+        na[u] = row_has_scale ? __ldg(sfa_row + static_cast<size_t>(kq) * p.sfa_ld) : 0.0f;           \
+        nl[u] = __ldg(sfb_lo + kq);                                                                   \
+        nh[u] = (BN % 128 == 0) ? 0.0f : __ldg(sfb_hi + kq);                                          \
+    }
+            FG8_LOAD_SCALE_GROUP(0)
+            int w = 0;
+            for (int kg = 0; kg < p.KB && w == 0; kg += SCALE_GROUP) {
+                float s_lo[SCALE_GROUP], s_hi[SCALE_GROUP];
 #pragma unroll
-            for (int q = 0; q < SCALE_AHEAD; ++q) {
-                const int kq = q < p.KB ? q : p.KB - 1;
-                ra[q] = row_in ? __ldg(sfa_p + static_cast<size_t>(kq) * p.sfa_ld) : 0.0f;
-                rl[q] = __ldg(sfb_lo + kq);
-                rh[q] = __ldg(sfb_hi + kq);
-            }
-            for (int kb = 0; kb < p.KB; ++kb) {
-                const float s_lo = ra[0] * rl[0];
-                const float s_hi = ra[0] * rh[0];
-#pragma unroll
-                for (int q = 0; q + 1 < SCALE_AHEAD; ++q) {
-                    ra[q] = ra[q + 1];
-                    rl[q] = rl[q + 1];
-                    rh[q] = rh[q + 1];
+                for (int u = 0; u < SCALE_GROUP; ++u) {
+                    s_lo[u] = na[u] * nl[u];
+                    s_hi[u] = (BN % 128 == 0) ? s_lo[u] : na[u] * nh[u];
                 }
-                {
-                    const int kq = kb + SCALE_AHEAD < p.KB ? kb + SCALE_AHEAD : p.KB - 1;
-                    ra[SCALE_AHEAD - 1] = row_in ? __ldg(sfa_p + static_cast<size_t>(kq) * p.sfa_ld) : 0.0f;
-                    rl[SCALE_AHEAD - 1] = __ldg(sfb_lo + kq);
-                    rh[SCALE_AHEAD - 1] = __ldg(sfb_hi + kq);
+                if (kg + SCALE_GROUP < p.KB) {
+                    FG8_LOAD_SCALE_GROUP(kg + SCALE_GROUP)
                 }
-                int w = 0;
-                if (lane == 0) w = wait_bar(&tfull[buf], bphase, limit, abort_flag);
-                w = __shfl_sync(0xffffffffu, w, 0);
-                if (w) {
-                    if (w == 2 && lane == 0) record_error(p.status, ERR_TIMEOUT, ROLE_EPILOGUE);
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-                const uint32_t tbase = tmem_base + lane_base + static_cast<uint32_t>(buf * S::ACC_STRIDE);
-                // Read the block's partial sums in batches of LB chunks (one
-                // tcgen05.wait::ld per batch), then scale and accumulate.
+#undef FG8_LOAD_SCALE_GROUP
 #pragma unroll
-                for (int i0 = 0; i0 < CPW; i0 += LB) {
-                    uint32_t r[LB][16];
+                for (int u = 0; u < SCALE_GROUP; ++u) {
+                    if (kg + u >= p.KB) break;
+                    if (lane == 0) w = wait_bar(&tfull[buf], bphase, limit, abort_flag);
+                    w = __shfl_sync(0xffffffffu, w, 0);
+                    if (w) break;
+                    ptx::tc_fence_after();
+                    const uint32_t tbase = tmem_base + lane_base + static_cast<uint32_t>(buf * S::ACC_STRIDE);
+                    // Software pipeline over batches of PB chunks: the TMEM loads of
+                    // batch q + 1 are in flight while batch q is scaled and added
+                    // (tcgen05.wait::ld waits for all of a thread's loads, so only
+                    // one batch is ever outstanding), and the accumulator is released
+                    // to the MMA issuers as soon as its last batch is in registers.
+                    uint32_t r[2][PB][16];
 #pragma unroll
-                    for (int b = 0; b < LB; ++b) {
-                        const int c = chunk0 + i0 + b;
-                        if (i0 + b < CPW && c < NC) ptx::tmem_ld16(tbase + static_cast<uint32_t>(c * 16), r[b]);
+                    for (int b = 0; b < PB; ++b) {
+                        const int c = chunk0 + b;
+                        if (b < CPW && c < NC) ptx::tmem_ld16(tbase + static_cast<uint32_t>(c * 16), r[0][b]);
                     }
                     ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int b = 0; b < LB; ++b) ptx::reg_fence(r[b]);
+                    for (int b = 0; b < PB; ++b) ptx::reg_fence(r[0][b]);
+                    if (NBATCH == 1) {
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if constexpr (PAIR) ptx::mbar_arrive_cluster(tempty_peer0 + static_cast<uint32_t>(buf * 8));
+                            else ptx::mbar_arrive(&tempty[buf]);
+                        }
+                    }
 #pragma unroll
-                    for (int b = 0; b < LB; ++b) {
-                        const int i = i0 + b;
-                        const int c = chunk0 + i;
-                        if (i < CPW && c < NC) {
-                            const float sc = (n0 + c * 16 >= split_col) ? s_hi : s_lo;
-                            const float2 sc2 = make_float2(sc, sc);
+                    for (int q = 0; q < NBATCH; ++q) {
+                        if (q + 1 < NBATCH) {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                const float2 v = make_float2(__uint_as_float(r[b][2 * j]), __uint_as_float(r[b][2 * j + 1]));
-                                acc[i < CPW ? i : 0][j] = __ffma2_rn(v, sc2, acc[i < CPW ? i : 0][j]);
+                            for (int b = 0; b < PB; ++b) {
+                                const int c = chunk0 + (q + 1) * PB + b;
+                                if ((q + 1) * PB + b < CPW && c < NC)
+                                    ptx::tmem_ld16(tbase + static_cast<uint32_t>(c * 16), r[(q + 1) & 1][b]);
+                            }
+                        }
+#pragma unroll
+                        for (int b = 0; b < PB; ++b) {
+                            const int i = q * PB + b;
+                            const int c = chunk0 + i;
+                            if (i < CPW && c < NC) {
+                                const float sc = (BN % 128 == 0) ? s_lo[u] : (((hi_mask >> i) & 1u) ? s_hi[u] : s_lo[u]);
+                                const float2 sc2 = make_float2(sc, sc);
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    const float2 v = make_float2(__uint_as_float(r[q & 1][b][2 * j]),
+                                                                 __uint_as_float(r[q & 1][b][2 * j + 1]));
+                                    acc[i < CPW ? i : 0][j] = __ffma2_rn(v, sc2, acc[i < CPW ? i : 0][j]);
+                                }
+                            }
+                        }
+                        if (q + 1 < NBATCH) {
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int b = 0; b < PB; ++b) ptx::reg_fence(r[(q + 1) & 1][b]);
+                            if (q + 2 == NBATCH) {
+                                // Every partial sum of this K block is in registers.
+                                ptx::tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) {
+                                    if constexpr (PAIR) ptx::mbar_arrive_cluster(tempty_peer0 + static_cast<uint32_t>(buf * 8));
+                                    else ptx::mbar_arrive(&tempty[buf]);
+                                }
                             }
                         }
                     }
-                }
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    if constexpr (PAIR) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_addr(&tempty[buf]), 0));
-                    else ptx::mbar_arrive(&tempty[buf]);
-                }
-                if (++buf == S::NBUF) {
-                    buf = 0;
-                    bphase ^= 1u;
+                    if (++buf == S::NBUF) {
+                        buf = 0;
+                        bphase ^= 1u;
+                    }
                 }
             }
-            if (!ok) break;
+            if (w) {
+                if (w == 2 && lane == 0) record_error(p.status, ERR_TIMEOUT, ROLE_EPILOGUE);
+                ok = false;
+                break;
+            }
 
             // ---- epilogue: BF16 (round to nearest even), rows that may be written only ----
             bool row_ok;
             if (p.layout == LAYOUT_NORMAL) {
-                row_ok = row_in;
+                row_ok = row < p.rows;
             } else if (p.layout == LAYOUT_CONTIGUOUS) {
-                row_ok = row_in && __ldg(p.m_indices + row) == t.g;
+                row_ok = row < p.rows && __ldg(p.m_indices + row) == t.g;
             } else {
                 int mm = __ldg(p.masked_m + t.g);
                 mm = mm > p.rows ? p.rows : mm;
                 row_ok = row < mm;
             }
             const uint32_t rows_mask = __ballot_sync(0xffffffffu, row_ok);
-            __nv_bfloat16* Dg = p.D + (p.layout == LAYOUT_MASKED ? static_cast<size_t>(t.g) * p.rows * p.N : 0);
+            if (rows_mask == 0u) continue;
             const int warp_row0 = t.row0 + quarter * 32;
-            if (rows_mask != 0u) {
+            const int d_g = p.layout == LAYOUT_MASKED ? t.g : 0;
+            // The staging slots may still be read by this warp's stores of the
+            // previous tile.
+            if (lane == 0) ptx::bulk_wait_group_read<0>();
+            __syncwarp();
+            const int sw = (lane >> 2) & 1;
+            // The D tensor map clips rows >= its row count and columns >= N, so a
+            // warp whose rows are all writable, or (normal layout) whose only
+            // unwritable rows lie past M, stores whole 32 x 16 pieces by TMA.
+            const bool bulk = rows_mask == 0xffffffffu || p.layout == LAYOUT_NORMAL;
+            if (bulk) {
 #pragma unroll
-                for (int i = 0; i < CPW; i += 2) {
-                    const int c0 = chunk0 + i;
-                    if (c0 >= NC) break;
-                    const bool has1 = (i + 1 < CPW) && (c0 + 1 < NC);
-                    uint8_t* myrow = stg + lane * EPI_PITCH;
-                    {
-                        uint4 v0, v1;
-                        v0.x = pack_bf16x2(acc[i][0].x, acc[i][0].y);
-                        v0.y = pack_bf16x2(acc[i][1].x, acc[i][1].y);
-                        v0.z = pack_bf16x2(acc[i][2].x, acc[i][2].y);
-                        v0.w = pack_bf16x2(acc[i][3].x, acc[i][3].y);
-                        v1.x = pack_bf16x2(acc[i][4].x, acc[i][4].y);
-                        v1.y = pack_bf16x2(acc[i][5].x, acc[i][5].y);
-                        v1.z = pack_bf16x2(acc[i][6].x, acc[i][6].y);
-                        v1.w = pack_bf16x2(acc[i][7].x, acc[i][7].y);
-                        *reinterpret_cast<uint4*>(myrow) = v0;
-                        *reinterpret_cast<uint4*>(myrow + 16) = v1;
+                for (int i = 0; i < CPW; ++i) {
+                    const int c = chunk0 + i;
+                    if (c >= NC || n0 + c * 16 >= p.N) break;
+                    uint8_t* piece = stg + (i & 1) * EPI_SLOT_BYTES;
+                    if (i >= EPI_SLOTS) {
+                        if (lane == 0) ptx::bulk_wait_group_read<EPI_SLOTS - 1>();
+                        __syncwarp();
                     }
-                    if (has1) {
-                        const int i1 = (i + 1) < CPW ? i + 1 : i;
-                        uint4 v0, v1;
-                        v0.x = pack_bf16x2(acc[i1][0].x, acc[i1][0].y);
-                        v0.y = pack_bf16x2(acc[i1][1].x, acc[i1][1].y);
-                        v0.z = pack_bf16x2(acc[i1][2].x, acc[i1][2].y);
-                        v0.w = pack_bf16x2(acc[i1][3].x, acc[i1][3].y);
-                        v1.x = pack_bf16x2(acc[i1][4].x, acc[i1][4].y);
-                        v1.y = pack_bf16x2(acc[i1][5].x, acc[i1][5].y);
-                        v1.z = pack_bf16x2(acc[i1][6].x, acc[i1][6].y);
-                        v1.w = pack_bf16x2(acc[i1][7].x, acc[i1][7].y);
-                        *reinterpret_cast<uint4*>(myrow + 32) = v0;
-                        *reinterpret_cast<uint4*>(myrow + 48) = v1;
-                    }
+                    *reinterpret_cast<uint4*>(piece + lane * 32 + (0 ^ sw) * 16) = pack_bf16x8(acc[i], 0);
+                    *reinterpret_cast<uint4*>(piece + lane * 32 + (1 ^ sw) * 16) = pack_bf16x8(acc[i], 1);
+                    ptx::fence_proxy_async_smem();
                     __syncwarp();
-                    const int units = has1 ? 4 : 2;     // 16-byte units per staged row
-                    const int col_base = n0 + c0 * 16;
-                    for (int q = lane; q < 32 * units; q += 32) {
-                        const int r = q / units;
-                        const int u = q - r * units;
-                        const int gcol = col_base + u * 8;
-                        if (((rows_mask >> r) & 1u) && gcol < p.N) {
-                            const uint4 v = *reinterpret_cast<const uint4*>(stg + r * EPI_PITCH + u * 16);
-                            *reinterpret_cast<uint4*>(Dg + static_cast<size_t>(warp_row0 + r) * p.N + gcol) = v;
+                    if (lane == 0) {
+                        ptx::tma_store_3d(&tmD, piece, n0 + c * 16, warp_row0, d_g);
+                        ptx::bulk_commit_group();
+                    }
+                }
+            } else {
+                __nv_bfloat16* Dg = p.D + static_cast<size_t>(d_g) * p.rows * p.N;
+#pragma unroll
+                for (int i = 0; i < CPW; ++i) {
+                    const int c = chunk0 + i;
+                    if (c >= NC || n0 + c * 16 >= p.N) break;
+                    uint8_t* piece = stg;
+                    *reinterpret_cast<uint4*>(piece + lane * 32 + (0 ^ sw) * 16) = pack_bf16x8(acc[i], 0);
+                    *reinterpret_cast<uint4*>(piece + lane * 32 + (1 ^ sw) * 16) = pack_bf16x8(acc[i], 1);
+                    __syncwarp();
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int u = lane + 32 * q;     // 16-byte unit: row u / 2, half u % 2
+                        const int r = u >> 1;
+                        const int h = u & 1;
+                        if ((rows_mask >> r) & 1u) {
+                            const uint4 v = *reinterpret_cast<const uint4*>(piece + r * 32 + (h ^ ((r >> 2) & 1)) * 16);
+                            *reinterpret_cast<uint4*>(Dg + static_cast<size_t>(warp_row0 + r) * p.N + n0 + c * 16 + h * 8) = v;
                         }
                     }
                     __syncwarp();
                 }
             }
         }
+        // Every bulk store of this warp must be complete before the CTA exits.
+        if (lane == 0) ptx::bulk_wait_group<0>();
     }
 
     __syncwarp();

@@ -18,12 +18,12 @@ constexpr int kMaxDynamicSmem = 232448;
 // register split is safe only at exactly REGS_LAUNCH) and raises the kernel's
 // shared-memory limit.  Defined in gemm_inst.cu, one block width per object.
 template <int BN, bool PAIR>
-cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p, int grid,
-                        size_t smem_bytes, cudaStream_t stream);
+cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD, const GemmParams& p,
+                        int grid, size_t smem_bytes, cudaStream_t stream);
 
 template <int BN, bool PAIR>
-cudaError_t launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p, int grid,
-                             size_t smem_bytes, cudaStream_t stream) {
+cudaError_t launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
+                             const GemmParams& p, int grid, size_t smem_bytes, cudaStream_t stream) {
     static std::atomic<unsigned long long> attr_set{0};
     static std::atomic<int> max_clusters[64];   // per device, 0 = not queried yet
     int dev = 0;
@@ -68,20 +68,20 @@ cudaError_t launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, con
         }
         if (grid > 2 * mc) cfg.gridDim.x = static_cast<unsigned>(2 * mc);
     }
-    return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, p);
+    return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmD, p);
 }
 
 #define FG8_DEFINE_LAUNCH_ONE(BN, PAIR)                                                                        \
     template <>                                                                                                \
-    cudaError_t launch_gemm<BN, PAIR>(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,     \
-                                      int grid, size_t smem_bytes, cudaStream_t stream) {                      \
-        return launch_gemm_impl<BN, PAIR>(tmA, tmB, p, grid, smem_bytes, stream);                              \
+    cudaError_t launch_gemm<BN, PAIR>(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,  \
+                                      const GemmParams& p, int grid, size_t smem_bytes, cudaStream_t stream) { \
+        return launch_gemm_impl<BN, PAIR>(tmA, tmB, tmD, p, grid, smem_bytes, stream);                         \
     }
 
 #define FG8_DECLARE_LAUNCH_ONE(BN, PAIR)                                                                       \
     template <>                                                                                                \
-    cudaError_t launch_gemm<BN, PAIR>(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,     \
-                                      int grid, size_t smem_bytes, cudaStream_t stream);
+    cudaError_t launch_gemm<BN, PAIR>(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,  \
+                                      const GemmParams& p, int grid, size_t smem_bytes, cudaStream_t stream);
 
 // Block widths 16..256; CTA pairs from 32 (each CTA loads at least 16 B rows).
 #define FG8_FOR_EACH_BN(X) \

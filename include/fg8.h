@@ -40,6 +40,14 @@
 #include <stddef.h>
 #include <stdint.h>
 
+/* The library is built with hidden symbol visibility; only the entry points
+ * declared here (marked FG8_API) are exported. */
+#if defined(__GNUC__)
+#define FG8_API __attribute__((visibility("default")))
+#else
+#define FG8_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -57,10 +65,10 @@ typedef enum {
 } fg_status;
 
 /* Human-readable name of a status code (static string). */
-const char* fg_status_string(int status);
+FG8_API const char* fg_status_string(int status);
 
 /* Library version, e.g. "fg8 0.1.0 sm_100a". */
-const char* fg_version(void);
+FG8_API const char* fg_version(void);
 
 /*
  * Normal GEMM, D = A . B^T with fine-grained scales.
@@ -74,7 +82,7 @@ const char* fg_version(void);
  *   D   [M, N]   bf16, row-major (row stride N elements), fully overwritten
  * M == 0 is a no-op.  Returns FG_OK or an error code.
  */
-fg_status fg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* D, int M,
+FG8_API fg_status fg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* D, int M,
                          int N, int K, fg_stream_t stream);
 
 /*
@@ -95,7 +103,7 @@ fg_status fg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const f
  * is not -1 unless the whole block is padding; rows that break this are left
  * unwritten.
  */
-fg_status fg_m_grouped_fp8_gemm_nt_contiguous(const void* A, const float* sfa, const void* B,
+FG8_API fg_status fg_m_grouped_fp8_gemm_nt_contiguous(const void* A, const float* sfa, const void* B,
                                               const float* sfb, void* D, const int* m_indices, int M_tot,
                                               int N, int K, int G, fg_stream_t stream);
 
@@ -111,7 +119,7 @@ fg_status fg_m_grouped_fp8_gemm_nt_contiguous(const void* A, const float* sfa, c
  *   expected_m: host-side hint of the typical masked_m used to pick the tile
  *            shape (0 = M_max).  It never changes the result.
  */
-fg_status fg_m_grouped_fp8_gemm_nt_masked(const void* A, const float* sfa, const void* B, const float* sfb,
+FG8_API fg_status fg_m_grouped_fp8_gemm_nt_masked(const void* A, const float* sfa, const void* B, const float* sfb,
                                           void* D, const int* masked_m, int G, int M_max, int N, int K,
                                           int expected_m, fg_stream_t stream);
 
@@ -119,25 +127,25 @@ fg_status fg_m_grouped_fp8_gemm_nt_masked(const void* A, const float* sfa, const
  * set_num_sms / get_num_sms).  Process-global.  Default: the device's SM
  * count (or the FG_NUM_SMS environment variable).  fg_set_num_sms accepts
  * 1 .. device SM count and returns FG_ERR_INVALID_ARG otherwise. */
-int fg_get_num_sms(void);
-fg_status fg_set_num_sms(int n);
+FG8_API int fg_get_num_sms(void);
+FG8_API fg_status fg_set_num_sms(int n);
 
 /* Row alignment of each expert segment in the contiguous layout (csdn page,
  * "实用工具": get_m_alignment_for_contiguous_layout).  Returns 128, the row
  * block of the kernels. */
-int fg_get_m_alignment_for_contiguous_layout(void);
+FG8_API int fg_get_m_alignment_for_contiguous_layout(void);
 
 /* Smallest n' >= n with n' * elem_bytes a multiple of 16 bytes, the TMA
  * stride rule (csdn page, "实用工具": get_tma_aligned_size).  elem_bytes must
  * divide 16; returns 0 otherwise. */
-size_t fg_get_tma_aligned_size(size_t n, size_t elem_bytes);
+FG8_API size_t fg_get_tma_aligned_size(size_t n, size_t elem_bytes);
 
 /* Scale layout transform (csdn page, "实用工具": get_col_major_tma_aligned_tensor).
  *   in  [G][M][KB] fp32 row-major (device)
  *   out [G][KB][M_pad] fp32 (device), M_pad = fg_get_tma_aligned_size(M, 4):
  *       out[g][kb][m] = in[g][m][kb] for m < M, 0 for M <= m < M_pad.
  * Both pointers 16-byte aligned (in: 4).  Runs one small kernel on stream. */
-fg_status fg_transform_sfa_to_tma_layout(const float* in, float* out, int G, int M, int KB, fg_stream_t stream);
+FG8_API fg_status fg_transform_sfa_to_tma_layout(const float* in, float* out, int G, int M, int KB, fg_stream_t stream);
 
 /* Activation quantiser, the step that prepares A for the GEMMs (fine-grained
  * scaling, chujupifa.com "机器之心报道", opening summary; the scale layout of
@@ -152,27 +160,27 @@ fg_status fg_transform_sfa_to_tma_layout(const float* in, float* out, int G, int
  *       (written, rows M .. M_pad-1 set to 0): the scale layout the GEMMs read.
  * K must be a positive multiple of 128; x, q and sfa 16-byte aligned.  M == 0
  * is a no-op.  Runs one kernel on stream. */
-fg_status fg_quantize_fp8_activations(const void* x, int x_is_bf16, void* q, float* sfa, int M, int K,
+FG8_API fg_status fg_quantize_fp8_activations(const void* x, int x_is_bf16, void* q, float* sfa, int M, int K,
                                       fg_stream_t stream);
 
 /* Reads and clears this device's status word after synchronising `stream`.
  * *code_out = 0 when no kernel recorded an error since the last call, else
  * FG_ERR_TIMEOUT; *detail_out (may be NULL) = (block << 8) | role of the
  * first failure (role 1 = TMA producer, 2 = MMA issuer, 3 = epilogue). */
-fg_status fg_get_last_device_status(fg_stream_t stream, int* code_out, int* detail_out);
+FG8_API fg_status fg_get_last_device_status(fg_stream_t stream, int* code_out, int* detail_out);
 
 /* Upper bound, in nanoseconds, on any single pipeline wait inside the GEMM
  * kernels (default 1e9 = 1 s; FG_WAIT_LIMIT_NS overrides at load).  A wait
  * that runs past it makes the kernel record FG_ERR_TIMEOUT, drain its copies
  * in flight, release tensor memory and return: it never hangs the GPU.
  * Values below 1000 are rejected. */
-fg_status fg_set_wait_limit_ns(unsigned long long ns);
-unsigned long long fg_get_wait_limit_ns(void);
+FG8_API fg_status fg_set_wait_limit_ns(unsigned long long ns);
+FG8_API unsigned long long fg_get_wait_limit_ns(void);
 
 /* The block width (BLOCK_N) the normal GEMM would use for (M, N, K) with the
  * current SM budget, negated when the tile runs on a pair of CTAs (256-row
  * tiles), or 0 for an unsupported shape.  Diagnostics. */
-int fg_query_block_n(int M, int N, int K);
+FG8_API int fg_query_block_n(int M, int N, int K);
 
 /* The launch plan a GEMM call of these sizes would use with the current SM
  * budget and environment (diagnostics; launches nothing, allocates nothing).
@@ -188,7 +196,7 @@ int fg_query_block_n(int M, int N, int K);
  *                shared memory when equal to *splits_out > 1)
  * Returns FG_ERR_INVALID_ARG for a bad layout, non-positive sizes or a NULL
  * output, FG_ERR_UNSUPPORTED when K % 128 != 0 or N % 16 != 0. */
-fg_status fg_query_plan(int layout, int rows, int N, int K, int G, int expected_m, int* kernel_out,
+FG8_API fg_status fg_query_plan(int layout, int rows, int N, int K, int G, int expected_m, int* kernel_out,
                         int* tile_n_out, int* pair_out, int* splits_out, int* cluster_out);
 
 /*
@@ -231,7 +239,7 @@ fg_status fg_query_plan(int layout, int rows, int N, int K, int G, int expected_
 #define FG_NO_ALLOC_MAX_N 262144
 #define FG_NO_ALLOC_PARTIAL_FLOATS (2u * 1024u * 1024u)
 #define FG_NO_ALLOC_SCRATCH_BYTES ((FG_NO_ALLOC_MAX_N / 128) * 4u + FG_NO_ALLOC_PARTIAL_FLOATS * 4u)
-fg_status fg_fp8_gemm_nt_small_m_no_alloc(const void* A, const float* sfa, const void* B, const float* sfb, void* D,
+FG8_API fg_status fg_fp8_gemm_nt_small_m_no_alloc(const void* A, const float* sfa, const void* B, const float* sfb, void* D,
                                           int M, int N, int K, fg_stream_t stream);
 
 #ifdef __cplusplus
