@@ -58,6 +58,8 @@ _SIG = {
     "fg_get_wait_limit_ns": (ctypes.c_ulonglong, []),
     "fg_query_block_n": (_I, [_I, _I, _I]),
     "fg_query_plan": (_I, [_I, _I, _I, _I, _I, _I] + [ctypes.POINTER(_I)] * 5),
+    "fg_jit_compile": (_I, [_I, _I, _I, ctypes.c_char_p, ctypes.c_size_t]),
+    "fg_jit_stats": (None, [ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "fg_fp8_gemm_nt_small_m_no_alloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "fg_quantize_fp8_activations": (_I, [_P, _I, _P, _P, _I, _I, _P]),
 }
@@ -329,3 +331,20 @@ def query_plan(layout: str, rows: int, N: int, K: int, G: int = 1, expected_m: i
     kernel, tile_n, pair, splits, cluster = (o.value for o in out)
     return {"kernel": "decode" if kernel == 1 else "tile", "tile_n": tile_n, "pair": bool(pair), "splits": splits,
             "cluster": cluster}
+
+
+def jit_compile(block_n: int, pair: bool, k_blocks: int) -> str:
+    """Compile (or find in the on-disk cache) the tile kernel specialised for
+    (block_n, pair, k_blocks) with NVRTC; returns the cubin's path.  Needs no
+    GPU.  The GEMMs use such kernels when FG_JIT=1 is set."""
+    buf = ctypes.create_string_buffer(4096)
+    _check(_lib.fg_jit_compile(int(block_n), 1 if pair else 0, int(k_blocks), buf, len(buf)), "jit_compile")
+    return buf.value.decode()
+
+
+def jit_stats() -> dict:
+    """Runtime specialisations compiled / read from the disk cache by this
+    process, and GEMM launches that ran a runtime-compiled kernel."""
+    c, d, n = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _lib.fg_jit_stats(ctypes.byref(c), ctypes.byref(d), ctypes.byref(n))
+    return {"compiled": c.value, "loaded_from_disk": d.value, "launches": n.value}

@@ -73,7 +73,7 @@ def build(force: bool = False, jobs: int = 0, verbose: bool = False) -> str:
         objs.append(o)
         cmds.append([nvcc(), *ARCH, *FLAGS, *ptxas, f"-DFG8_MT={mt}", "-c",
                      os.path.join(CSRC, "decode_inst.cu"), "-o", o])
-    for src in ["fg8_host.cu", "quant.cu"]:
+    for src in ["fg8_host.cu", "quant.cu", "jit.cu"]:
         o = os.path.join(BUILD, src.replace(".cu", ".o"))
         objs.append(o)
         cmds.append([nvcc(), *ARCH, *FLAGS, *ptxas, "-c", os.path.join(CSRC, src), "-o", o])

@@ -15,6 +15,7 @@
 
 #include "decode_launch.cuh"
 #include "fg8.h"
+#include "jit.h"
 #include "launch.cuh"
 
 namespace fg8 {
@@ -216,14 +217,48 @@ struct Choice {
     bool pair = false;
 };
 
-double estimate_cycles(bool pair, int bn, long long row_tiles, int N, int K, int num_sms, double hbm_bytes) {
+// ---- stream-K (normal layout) ----------------------------------------------------
+// When the tiles fill the units' last wave poorly, all but the last one or two
+// waves of tiles run whole and the (tile, K block) iterations of the rest are
+// split evenly over the units (see TileScheduler).  Used when that wave would
+// be less than 90 % full and every unit gets at least a quarter of a tile's K
+// blocks (so a tile is split over a few units at most).  FG_STREAMK=0 turns it
+// off.
+struct StreamKPlan {
+    bool on = false;
+    int dp_tiles = 0;
+    long long iters = 0;
+};
+
+StreamKPlan streamk_plan(long long tiles, int units, int KB) {
+    StreamKPlan sp;
+    const char* env = std::getenv("FG_STREAMK");
+    if ((env && std::atoi(env) == 0) || units <= 1 || tiles <= 0 || KB < 2) return sp;
+    const long long waves = (tiles + units - 1) / units;
+    const double fill = static_cast<double>(tiles) / static_cast<double>(waves * units);
+    if (fill >= 0.9) return sp;
+    const long long full_waves = tiles / units;
+    const long long dp = full_waves > 1 ? (full_waves - 1) * units : 0;
+    const long long iters = (tiles - dp) * KB;
+    if (iters * 4 < static_cast<long long>(units) * KB) return sp;   // pieces shorter than KB / 4
+    sp.on = true;
+    sp.dp_tiles = static_cast<int>(dp);
+    sp.iters = iters;
+    return sp;
+}
+
+double estimate_cycles(int layout, bool pair, int bn, long long row_tiles, int N, int K, int num_sms,
+                       double hbm_bytes) {
     const int KB = K / BK;
     const long long tiles = row_tiles * ((N + bn - 1) / bn);
     const int units = std::max(1, pair ? num_sms / 2 : num_sms);
-    const double waves = static_cast<double>((tiles + units - 1) / units);
+    double waves = static_cast<double>((tiles + units - 1) / units);
+    if (layout == LAYOUT_NORMAL && streamk_plan(tiles, units, KB).on)
+        waves = static_cast<double>(tiles) / units + 0.05;   // split iterations, plus the partial-sum exchange
     const int acc_stride = (bn + 31) / 32 * 32;
     const int nbuf = std::min(4, 512 / acc_stride);
-    const double per_kb = nbuf >= 4 ? 520.0 : (nbuf == 3 ? 600.0 : 700.0);
+    double per_kb = nbuf >= 4 ? 520.0 : (nbuf == 3 ? 600.0 : 700.0);
+    if (pair) per_kb *= 0.96;   // a pair's 256-row tile runs a few per cent faster than two 128-row tiles
     const double t_tiles = waves * (KB * per_kb + 2000.0);
     return std::max(t_tiles, hbm_bytes / 3300.0) + 2000.0;
 }
@@ -236,10 +271,8 @@ Choice choose_config(int layout, int rows, int groups, int valid_rows, int N, in
     const char* force_pair = std::getenv("FG_FORCE_PAIR");
     const int fbn = force ? std::atoi(force) : 0;
     const int fpair = force_pair ? std::atoi(force_pair) : -1;
-    // CTA pairs halve each SM's B loads, but on B200 their cross-CTA handshake
-    // costs more than it saves for every workload measured so far, so they run
-    // only on request (FG_FORCE_PAIR=1).
-    const bool pair_ok = fpair == 1 && num_sms >= 2 && !(layout == LAYOUT_CONTIGUOUS && rows / BM > MAX_PAIR_LIST);
+    // CTA pairs halve each SM's B loads; FG_FORCE_PAIR=0/1 forbids/forces them.
+    const bool pair_ok = fpair != 0 && num_sms >= 2 && !(layout == LAYOUT_CONTIGUOUS && rows / BM > MAX_PAIR_LIST);
     double best_t = 1e300;
     for (int pair = 0; pair <= 1; ++pair) {
         if (pair && !pair_ok) continue;
@@ -248,7 +281,7 @@ Choice choose_config(int layout, int rows, int groups, int valid_rows, int N, in
             if (fbn >= 16 && fbn <= 256 && fbn % 16 == 0 && bn != fbn) continue;
             const int tile_m = pair ? 2 * BM : BM;
             const long long row_tiles = static_cast<long long>(groups) * ((valid_rows + tile_m - 1) / tile_m);
-            const double t = estimate_cycles(pair, bn, std::max(1ll, row_tiles), N, K, num_sms, hbm_bytes);
+            const double t = estimate_cycles(layout, pair, bn, std::max(1ll, row_tiles), N, K, num_sms, hbm_bytes);
             if (t < best_t * 0.999 || (t <= best_t * 1.001 && (pair > (best.pair ? 1 : 0) || bn > best.bn))) {
                 if (t < best_t) best_t = t;
                 best.bn = bn;
@@ -266,7 +299,7 @@ int stage_bytes_for(int bn, bool pair) { return BM * BK + (pair ? bn / 2 : bn) *
 int choose_stages(int bn, bool pair) {
     const int sb = stage_bytes_for(bn, pair);
     int s = 8;
-    while (s > MAX_NBUF && gemm_smem_bytes(sb, s, pair) > static_cast<size_t>(kMaxDynamicSmem)) --s;
+    while (s > MAX_NBUF && gemm_smem_bytes(sb, s, pair) > static_cast<size_t>(kMaxDynamicSmem - kGemmStaticSmem)) --s;
     return s;
 }
 
@@ -535,6 +568,53 @@ int decode_max_rows() {
     return env ? std::atoi(env) : 128;
 }
 
+// Workspace of the stream-K partial sums and their flags, one per (device,
+// stream), grown on demand and kept for the life of the process (launches on
+// one stream run in order).  Flags hold the epoch of the launch that published
+// them: each launch takes a new epoch, so stale flags never match.
+struct StreamKWorkspace {
+    float* ws = nullptr;
+    size_t ws_bytes = 0;
+    unsigned* flags = nullptr;
+    size_t flag_count = 0;
+    unsigned epoch = 0;
+};
+std::map<std::pair<int, cudaStream_t>, StreamKWorkspace> g_sk;
+std::mutex g_sk_mutex;
+
+fg_status get_streamk_workspace(int dev, cudaStream_t stream, size_t ws_bytes, size_t flags, float** ws,
+                                unsigned** fl, unsigned* epoch) {
+    std::lock_guard<std::mutex> lk(g_sk_mutex);
+    StreamKWorkspace& w = g_sk[std::make_pair(dev, stream)];
+    if (w.ws_bytes < ws_bytes) {
+        if (w.ws) cudaFree(w.ws);
+        w.ws = nullptr;
+        w.ws_bytes = 0;
+        if (cudaMalloc(&w.ws, ws_bytes) != cudaSuccess) {
+            cudaGetLastError();
+            return FG_ERR_CUDA;
+        }
+        w.ws_bytes = ws_bytes;
+    }
+    if (w.flag_count < flags) {
+        if (w.flags) cudaFree(w.flags);
+        w.flags = nullptr;
+        w.flag_count = 0;
+        if (cudaMalloc(&w.flags, flags * sizeof(unsigned)) != cudaSuccess ||
+            cudaMemset(w.flags, 0, flags * sizeof(unsigned)) != cudaSuccess) {
+            cudaGetLastError();
+            return FG_ERR_CUDA;
+        }
+        w.flag_count = flags;
+        w.epoch = 0;
+    }
+    if (++w.epoch == 0) w.epoch = 1;
+    *ws = w.ws;
+    *fl = w.flags;
+    *epoch = w.epoch;
+    return FG_OK;
+}
+
 // Shared by the three GEMM kinds once their arguments are checked.
 fg_status run_gemm(int layout, const void* A, const float* sfa, const void* B, const float* sfb, void* D,
                    const int* m_indices, const int* masked_m, int rows, int N, int K, int G, int valid_rows_hint,
@@ -590,8 +670,24 @@ fg_status run_gemm(int layout, const void* A, const float* sfa, const void* B, c
                                                             : static_cast<long long>(a_groups) * p.num_m_tiles;
     const long long tiles = row_tiles * p.num_n_blocks;
     const int units = c.pair ? num_sms / 2 : num_sms;
-    const long long used = std::max<long long>(1, std::min<long long>(tiles, units));
+    long long used = std::max<long long>(1, std::min<long long>(tiles, units));
+    if (layout == LAYOUT_NORMAL) {
+        const StreamKPlan sp = streamk_plan(tiles, units, KB);
+        if (sp.on) {
+            used = units;
+            const size_t ctas = static_cast<size_t>(c.pair ? 2 * used : used);
+            int dev_id = 0;
+            cudaGetDevice(&dev_id);
+            st = get_streamk_workspace(dev_id, stream, ctas * BM * bn * sizeof(float), ctas * NUM_EPI_WARPS, &p.sk_ws,
+                                       &p.sk_flags, &p.sk_epoch);
+            if (st != FG_OK) return st;
+            p.sk = 1;
+            p.sk_dp_tiles = sp.dp_tiles;
+            p.sk_iters = sp.iters;
+        }
+    }
     const int grid = static_cast<int>(c.pair ? 2 * used : used);
+    if (jit_enabled() && jit_launch_gemm(bn, c.pair, ta, tb, td, p, grid, smem, stream) == FG_OK) return FG_OK;
     return launch_bn(bn, c.pair, ta, tb, td, p, grid, smem, stream);
 }
 

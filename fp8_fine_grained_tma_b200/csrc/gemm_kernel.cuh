@@ -40,9 +40,16 @@
 #pragma once
 
 #include <cuda_bf16.h>
-#include <cstdint>
+
+#include "rtc_compat.cuh"
 
 #include "ptx.cuh"
+
+// K blocks of the problem as a compile-time constant when the kernel is
+// compiled at run time for one shape (0: taken from the parameters).
+#ifndef FG8_KB_CT
+#define FG8_KB_CT 0
+#endif
 
 namespace fg8 {
 
@@ -72,6 +79,7 @@ constexpr int EPI_WARP_BYTES = EPI_SLOTS * EPI_SLOT_BYTES;
 // Scales are loaded by the promotion threads themselves, SCALE_GROUP K blocks
 // at a time, one group ahead of their use.
 constexpr int SCALE_GROUP = 2;
+constexpr int SCALE_PREFETCH = 8;                  // K blocks between the L1 prefetch of sfa and its load
 constexpr int A_TILE_BYTES = BM * BK;              // 16 KiB
 // Contiguous layout, CTA pairs: the 128-row blocks that start a pair tile are
 // listed in shared memory (one 16-bit block index each).
@@ -100,6 +108,18 @@ struct GemmParams {
     const int* masked_m;
     int* status;       // [0] = first error code, [1] = (block << 8) | role
     unsigned long long wait_limit_ns;
+    // Stream-K (normal layout): the first sk_dp_tiles tiles are processed whole,
+    // wave by wave; the (tile, K block) iterations of the remaining tiles are
+    // split evenly over the units.  sk_ws holds one FP32 partial tile slice per
+    // CTA ([grid][NC][128][16]), sk_flags the epoch of the last partial each
+    // promotion warp of each CTA published ([grid][8]); sk_epoch is this
+    // launch's (never 0).
+    int sk;                  // 1: stream-K on
+    int sk_dp_tiles;         // tiles processed whole before the split ones
+    long long sk_iters;      // (tiles - sk_dp_tiles) * KB
+    float* sk_ws;
+    unsigned* sk_flags;
+    unsigned sk_epoch;
 };
 
 __host__ __device__ constexpr int ceil_div_c(int a, int b) { return (a + b - 1) / b; }
@@ -147,6 +167,8 @@ struct TileInfo {
     int g;       // group of B / sfb (expert); for the masked layout also of A / D
     int row0;    // first row (within the group) of this CTA's 128-row slice of the tile
     int n_blk;
+    int kb0, kb1;      // K blocks [kb0, kb1) of the tile processed here (0, KB unless stream-K)
+    int sk_first;      // stream-K, kb0 > 0 and kb1 == KB: first unit whose partial this one adds
 };
 
 // Enumerates the tiles of this CTA (or CTA pair).  Every role builds its own
@@ -160,12 +182,92 @@ struct TileScheduler {
     const uint16_t* pair_list;         // contiguous layout with pairs
     int pair_count;
 
-    __device__ TileScheduler(int unit, int num_units, int rank_, const uint16_t* list, int count)
-        : next(unit), stride(num_units), rank(rank_), mg(0), mbase(0), mtiles(-1), mtiles_m(0), pair_list(list),
-          pair_count(count) {}
+    long long sk_lo, sk_cur;           // stream-K: this unit's iteration range [sk_lo, sk_hi), walked backwards
+    int unit_, units_;
+
+    __device__ TileScheduler(int unit, int num_units, int rank_, const uint16_t* list, int count) {
+        init(unit, num_units, rank_, list, count);
+    }
+    TileScheduler() = default;
+
+    __device__ void init(int unit, int num_units, int rank_, const uint16_t* list, int count) {
+        next = unit;
+        stride = num_units;
+        rank = rank_;
+        mg = 0;
+        mbase = 0;
+        mtiles = -1;
+        mtiles_m = 0;
+        pair_list = list;
+        pair_count = count;
+        sk_lo = 0;
+        sk_cur = 0;
+        unit_ = unit;
+        units_ = num_units;
+    }
+
+    // First iteration of unit u's stream-K range.
+    __device__ static long long sk_start(const GemmParams& p, int u, int units) {
+        return static_cast<long long>(u) * p.sk_iters / units;
+    }
+
+    // Raster-grouped tile order: tile index -> (row tile, column block).
+    __device__ static void raster(const GemmParams& p, int idx, int& m_tile, int& n_blk) {
+        const int per_group = p.raster_m * p.num_n_blocks;
+        const int grp = idx / per_group;
+        const int first_m = grp * p.raster_m;
+        const int gm = min(p.raster_m, p.num_m_tiles - first_m);
+        const int local = idx - grp * per_group;
+        m_tile = first_m + local % gm;
+        n_blk = local / gm;
+    }
 
     __device__ bool get(const GemmParams& p, TileInfo& t) {
         constexpr int TILE_M = PAIR ? 2 * BM : BM;
+        t.kb0 = 0;
+        t.kb1 = FG8_KB_CT > 0 ? FG8_KB_CT : p.KB;
+        t.sk_first = -1;
+        if (p.sk) {
+            // Whole tiles first (unit, unit + units, ... below sk_dp_tiles), then
+            // this unit's share of the split iterations, last piece first: a
+            // piece that ends inside its tile (its partial sum goes to the
+            // workspace) is done before the pieces that finish tiles.
+            if (next < p.sk_dp_tiles) {
+                const int idx = next;
+                next += stride;
+                int m_tile;
+                raster(p, idx, m_tile, t.n_blk);
+                t.row0 = m_tile * TILE_M + rank * BM;
+                t.g = 0;
+                return true;
+            }
+            if (next != 0x7fffffff) {   // entering the split part: set up the range
+                next = 0x7fffffff;
+                sk_lo = sk_start(p, unit_, units_);
+                sk_cur = sk_start(p, unit_ + 1, units_);
+            }
+            if (sk_cur <= sk_lo) return false;
+            const long long last = sk_cur - 1;
+            const int tile = static_cast<int>(last / p.KB);
+            const long long tile_start = static_cast<long long>(tile) * p.KB;
+            const long long b = max(sk_lo, tile_start);
+            t.kb0 = static_cast<int>(b - tile_start);
+            t.kb1 = static_cast<int>(sk_cur - tile_start);
+            sk_cur = b;
+            if (t.kb0 > 0 && t.kb1 == p.KB) {
+                // The unit holding this tile's first iteration: the largest u
+                // with sk_start(u) <= tile_start.
+                int u = static_cast<int>(tile_start * units_ / max(1ll, p.sk_iters));
+                while (u + 1 < units_ && sk_start(p, u + 1, units_) <= tile_start) ++u;
+                while (u > 0 && sk_start(p, u, units_) > tile_start) --u;
+                t.sk_first = u;
+            }
+            int m_tile;
+            raster(p, p.sk_dp_tiles + tile, m_tile, t.n_blk);
+            t.row0 = m_tile * TILE_M + rank * BM;
+            t.g = 0;
+            return true;
+        }
         if (p.layout == LAYOUT_MASKED) {
             const int idx = next;
             while (true) {
@@ -382,7 +484,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             while (w == 0 && sch.get(p, t)) {
                 const int a_g = p.layout == LAYOUT_MASKED ? t.g : 0;
                 const int b_row = t.n_blk * BN + rank * S::BNL;
-                for (int kb = 0; kb < p.KB; ++kb) {
+                for (int kb = t.kb0; kb < t.kb1; ++kb) {
                     w = wait_bar(&empty[stage], phase ^ 1u, limit, abort_flag);
                     if (w) break;
                     uint8_t* sa = stage_base + static_cast<size_t>(stage) * S::STAGE_BYTES;
@@ -442,7 +544,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int w = 0;
             int g = 0;
             while (w == 0 && sch.get(p, t)) {
-                for (int kb = 0; kb < p.KB; ++kb, ++g) {
+                for (int kb = t.kb0; kb < t.kb1; ++kb, ++g) {
                     if (g % NUM_MMA_WARPS == j) {
                         w = wait_bar(&tempty[buf], bphase ^ 1u, limit, abort_flag);
                         if (w) break;
@@ -501,12 +603,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint8_t* stg = epi_base + warp * EPI_WARP_BYTES;
         const uint32_t tempty_peer0 = PAIR ? ptx::mapa_shared(ptx::smem_addr(&tempty[0]), 0) : 0u;
 
-        TileScheduler<PAIR> sch(unit, num_units, rank, pair_list, pair_count);
+        // The tile sequence is only needed between tiles: lane 0 walks it with
+        // its state in shared memory and hands each tile to the warp by
+        // shuffles, which keeps the registers for the accumulators.
+        __shared__ TileScheduler<PAIR> sched_store[NUM_EPI_WARPS];
+        if (lane == 0) sched_store[warp].init(unit, num_units, rank, pair_list, pair_count);
         TileInfo t;
         int buf = 0;
         uint32_t bphase = 0;
         bool ok = true;
-        while (ok && sch.get(p, t)) {
+        while (ok) {
+            int has = 0;
+            if (lane == 0) has = sched_store[warp].get(p, t) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, has, 0)) break;
+            t.g = __shfl_sync(0xffffffffu, t.g, 0);
+            t.row0 = __shfl_sync(0xffffffffu, t.row0, 0);
+            t.n_blk = __shfl_sync(0xffffffffu, t.n_blk, 0);
+            t.kb0 = __shfl_sync(0xffffffffu, t.kb0, 0);
+            t.kb1 = __shfl_sync(0xffffffffu, t.kb1, 0);
+            t.sk_first = __shfl_sync(0xffffffffu, t.sk_first, 0);
             const int row = t.row0 + row_in_tile;
             const int n0 = t.n_blk * BN;
             // Scale block of this warpgroup's chunks: nb_lo for the first chunk,
@@ -554,22 +669,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         nl[u] = __ldg(sfb_lo + kq);                                                                   \
         nh[u] = (BN % 128 == 0) ? 0.0f : __ldg(sfb_hi + kq);                                          \
     }
-            FG8_LOAD_SCALE_GROUP(0)
+            if (row_has_scale) {
+                for (int kq = t.kb0 + SCALE_GROUP; kq < min(t.kb1, t.kb0 + SCALE_PREFETCH); ++kq)
+                    ptx::prefetch_l1(sfa_row + static_cast<size_t>(kq) * p.sfa_ld);
+            }
+            FG8_LOAD_SCALE_GROUP(t.kb0)
             int w = 0;
-            for (int kg = 0; kg < p.KB && w == 0; kg += SCALE_GROUP) {
+            // A kernel compiled for one shape knows the K blocks of a whole tile.
+            const int kb_end = (FG8_KB_CT > 0 && !p.sk) ? FG8_KB_CT : t.kb1;
+            for (int kg = t.kb0; kg < kb_end && w == 0; kg += SCALE_GROUP) {
                 float s_lo[SCALE_GROUP], s_hi[SCALE_GROUP];
 #pragma unroll
                 for (int u = 0; u < SCALE_GROUP; ++u) {
                     s_lo[u] = na[u] * nl[u];
                     s_hi[u] = (BN % 128 == 0) ? s_lo[u] : na[u] * nh[u];
                 }
-                if (kg + SCALE_GROUP < p.KB) {
+                if (kg + SCALE_GROUP < kb_end) {
                     FG8_LOAD_SCALE_GROUP(kg + SCALE_GROUP)
+                }
+                // sfa is a new 512-byte slice per K block: bring the slices of
+                // SCALE_PREFETCH K blocks ahead into L1 so that the loads above
+                // find them there instead of waiting on L2 behind the operand
+                // traffic.
+                if (row_has_scale) {
+#pragma unroll
+                    for (int u = 0; u < SCALE_GROUP; ++u)
+                        if (kg + SCALE_PREFETCH + u < kb_end)
+                            ptx::prefetch_l1(sfa_row + static_cast<size_t>(kg + SCALE_PREFETCH + u) * p.sfa_ld);
                 }
 #undef FG8_LOAD_SCALE_GROUP
 #pragma unroll
                 for (int u = 0; u < SCALE_GROUP; ++u) {
-                    if (kg + u >= p.KB) break;
+                    if (kg + u >= kb_end) break;
                     if (lane == 0) w = wait_bar(&tfull[buf], bphase, limit, abort_flag);
                     w = __shfl_sync(0xffffffffu, w, 0);
                     if (w) break;
@@ -647,6 +778,81 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (w == 2 && lane == 0) record_error(p.status, ERR_TIMEOUT, ROLE_EPILOGUE);
                 ok = false;
                 break;
+            }
+
+            // ---- stream-K: publish a partial sum, or add the earlier ones ----
+            if (t.kb1 < p.KB) {
+                // This piece ends inside its tile: store its FP32 partial sum in
+                // this CTA's workspace slice and publish it with the epoch.
+                float* ws = p.sk_ws + static_cast<size_t>(blockIdx.x) * NC * BM * 16;
+#pragma unroll
+                for (int i = 0; i < CPW; ++i) {
+                    const int c = chunk0 + i;
+                    if (c >= NC) break;
+                    float4* dst = reinterpret_cast<float4*>(ws + (static_cast<size_t>(c) * BM + row_in_tile) * 16);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        __stcg(dst + q, make_float4(acc[i][2 * q].x, acc[i][2 * q].y, acc[i][2 * q + 1].x,
+                                                    acc[i][2 * q + 1].y));
+                }
+                // Each warp publishes its own rows x columns: the warp of the same
+                // position in the finishing CTA waits for exactly this flag, so no
+                // warp waits on another warp of its own CTA.
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) ptx::st_release_gpu(p.sk_flags + blockIdx.x * NUM_EPI_WARPS + warp, p.sk_epoch);
+                continue;
+            }
+            if (t.sk_first >= 0) {
+                // This piece finishes its tile: add the partial sums of the units
+                // that did its first K blocks, in unit order (deterministic).
+                const int my_unit = PAIR ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+                for (int u = t.sk_first; u < my_unit && ok; ++u) {
+                    // A unit with no split iterations published nothing.
+                    if (TileScheduler<PAIR>::sk_start(p, u, num_units) == TileScheduler<PAIR>::sk_start(p, u + 1, num_units))
+                        continue;
+                    const int cta = PAIR ? 2 * u + rank : u;
+                    const unsigned* flag = p.sk_flags + cta * NUM_EPI_WARPS + warp;
+                    int w2 = 0;
+                    if (lane == 0) {
+                        const uint64_t t0 = ptx::globaltimer();
+                        while (ptx::ld_acquire_gpu(flag) != p.sk_epoch) {
+                            if (*abort_flag) {
+                                w2 = 1;
+                                break;
+                            }
+                            if (ptx::globaltimer() - t0 > limit) {
+                                *abort_flag = 1;
+                                w2 = 2;
+                                break;
+                            }
+                        }
+                    }
+                    w2 = __shfl_sync(0xffffffffu, w2, 0);
+                    if (w2) {
+                        if (w2 == 2 && lane == 0) record_error(p.status, ERR_TIMEOUT, ROLE_EPILOGUE);
+                        ok = false;
+                        break;
+                    }
+                    (void)ptx::ld_acquire_gpu(flag);   // every lane acquires the published partial
+                    const float* ws = p.sk_ws + static_cast<size_t>(cta) * NC * BM * 16;
+#pragma unroll
+                    for (int i = 0; i < CPW; ++i) {
+                        const int c = chunk0 + i;
+                        if (c >= NC) break;
+                        const float4* src =
+                            reinterpret_cast<const float4*>(ws + (static_cast<size_t>(c) * BM + row_in_tile) * 16);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 v = __ldcg(src + q);
+                            acc[i][2 * q].x += v.x;
+                            acc[i][2 * q].y += v.y;
+                            acc[i][2 * q + 1].x += v.z;
+                            acc[i][2 * q + 1].y += v.w;
+                        }
+                    }
+                }
+                if (!ok) break;
             }
 
             // ---- epilogue: BF16 (round to nearest even), rows that may be written only ----

@@ -10,8 +10,12 @@
 
 namespace fg8 {
 
-// Largest dynamic shared memory a CTA may request on sm_100 (227 KiB).
+// Largest shared memory (static + dynamic) a CTA may use on sm_100 (227 KiB).
 constexpr int kMaxDynamicSmem = 232448;
+// Static shared memory of the GEMM kernel (the promotion warps' tile
+// schedulers), reserved out of kMaxDynamicSmem when the stages are sized.
+constexpr int kGemmStaticSmem = 1024;
+static_assert(NUM_EPI_WARPS * sizeof(TileScheduler<true>) <= kGemmStaticSmem, "static shared memory");
 
 // Launches fg8_gemm_kernel<BN, PAIR> on `grid` CTAs (PAIR: clusters of two).
 // On first use per device it checks the build's register count (the in-kernel
@@ -36,7 +40,9 @@ cudaError_t launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, con
         e = cudaFuncGetAttributes(&fa, kernel);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != REGS_LAUNCH) return cudaErrorInvalidDeviceFunction;
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynamicSmem);
+        if (fa.sharedSizeBytes > static_cast<size_t>(kGemmStaticSmem)) return cudaErrorInvalidDeviceFunction;
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMaxDynamicSmem - static_cast<int>(fa.sharedSizeBytes));
         if (e != cudaSuccess) return e;
         attr_set.fetch_or(bit);
     }
@@ -60,7 +66,7 @@ cudaError_t launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, con
         int mc = max_clusters[dev & 63].load();
         if (mc == 0) {
             cudaLaunchConfig_t q = cfg;
-            q.dynamicSmemBytes = kMaxDynamicSmem;
+            q.dynamicSmemBytes = kMaxDynamicSmem - kGemmStaticSmem;
             e = cudaOccupancyMaxActiveClusters(&mc, kernel, &q);
             if (e != cudaSuccess) return e;
             if (mc <= 0) return cudaErrorInvalidConfiguration;

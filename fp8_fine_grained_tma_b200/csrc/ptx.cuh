@@ -6,8 +6,7 @@
 // wind down instead of hanging the GPU.
 #pragma once
 
-#include <cstdint>
-#include <cuda.h>
+#include "rtc_compat.cuh"
 
 namespace fg8 {
 namespace ptx {
@@ -127,6 +126,11 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
     return p;
+}
+
+// Bring the line holding `p` into L1 (no register, no completion to wait for).
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -367,6 +371,19 @@ __device__ __forceinline__ unsigned atom_inc_acq_rel_gpu(unsigned* addr, unsigne
     unsigned old;
     asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(limit) : "memory");
     return old;
+}
+
+// Store with release semantics at GPU scope: orders this thread's earlier
+// writes (and, through a preceding CTA barrier, those of the CTA) before it.
+__device__ __forceinline__ void st_release_gpu(unsigned* addr, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+
+// Load with acquire semantics at GPU scope.
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* addr) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+    return v;
 }
 
 // Named barrier among `count` threads (a multiple of 32) of the CTA.

@@ -8,8 +8,8 @@
 // get_col_major_tma_aligned_tensor (deepseek.csdn.net "DeepGEMM：简洁、高效…",
 // section "实用工具").  Per block:
 //   scale = max(amax, 1e-4) / 448        (FP32; 448 = largest finite E4M3)
-//   q     = E4M3(x / scale)              (FP32 division, round to nearest even,
-//                                         saturating at +-448)
+//   q     = E4M3(x / scale)              (the FP32 quotient rounded to nearest
+//                                         even, then to E4M3, saturating at +-448)
 // so the block's largest magnitude lands on 448.  The 1e-4 floor keeps an
 // all-zero block finite.
 //
@@ -40,6 +40,27 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
     f.z = __uint_as_float(u.y << 16);
     f.w = __uint_as_float(u.y & 0xFFFF0000u);
     return f;
+}
+
+// x / b rounded to nearest even, given y = the correctly rounded reciprocal
+// of b.  Markstein's method (P. Markstein, "IA-64 and Elementary Functions",
+// 2000): with the residual r = x - b q computed exactly by an FMA, q + r y
+// rounded once is the correctly rounded quotient when q is within one unit in
+// the last place of x / b.  x * y alone can be 1.5 units off, so one residual
+// step brings it within one unit and a second gives the correctly rounded
+// result.  Computed on |x| with the sign put back at the end, so that -0 / b
+// stays -0 (a residual step would turn it into +0).  Used for the per-element
+// quotients; valid for the normal scales and |x / b| <= 448 (plus rounding)
+// of the quantiser.  The tests check the codes bit for bit against IEEE
+// division on values within a few units of every E4M3 rounding boundary.
+__device__ __forceinline__ float div_rn(float x, float b, float y) {
+    const float a = fabsf(x);
+    float q = a * y;
+    float r = fmaf(-q, b, a);
+    q = fmaf(r, y, q);
+    r = fmaf(-q, b, a);
+    q = fmaf(r, y, q);
+    return copysignf(q, x);
 }
 
 // Four FP32 -> four E4M3 codes (round to nearest even, saturating), byte i = value i.
@@ -73,7 +94,9 @@ __global__ void __launch_bounds__(QTHREADS, 8) quantize_kernel(const T* __restri
             for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             if (b >= nblk) continue;   // warp-uniform
             const float scale = fmaxf(amax, 1e-4f) / 448.0f;
-            const uint32_t codes = to_e4m3x4(v[u].x / scale, v[u].y / scale, v[u].z / scale, v[u].w / scale);
+            const float rcp = __frcp_rn(scale);
+            const uint32_t codes = to_e4m3x4(div_rn(v[u].x, scale, rcp), div_rn(v[u].y, scale, rcp),
+                                             div_rn(v[u].z, scale, rcp), div_rn(v[u].w, scale, rcp));
             __stcs(reinterpret_cast<uint32_t*>(q + b * QBLK) + lane, codes);
             if (lane == 0) {
                 const long long m = b / KB;

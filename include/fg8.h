@@ -200,6 +200,31 @@ FG8_API fg_status fg_query_plan(int layout, int rows, int N, int K, int G, int e
                         int* tile_n_out, int* pair_out, int* splits_out, int* cluster_out);
 
 /*
+ * Runtime specialisation (the pages' library compiles its kernels at run time
+ * per shape and caches them on disk: chujupifa.com "机器之心报道", opening
+ * summary; deepseek.csdn.net "DeepGEMM：简洁、高效…", section "环境变量").
+ * With FG_JIT=1 in the environment, the normal GEMM's tile kernel is compiled
+ * with NVRTC for its block width, CTA pairing and K block count (a
+ * compile-time constant of the kernel), once per process, and the cubin is
+ * cached under FG_CACHE_DIR (default $HOME/.cache/fg8) for later processes.
+ * If NVRTC (libnvrtc.so.12), the kernel sources (next to the library, in
+ * csrc/) or a driver entry point is missing, the ahead-of-time kernel runs
+ * instead.
+ *
+ * fg_jit_compile: compiles (or finds in the cache) the specialisation for
+ *   block_n (16..256, multiple of 16), pair (0/1; block_n >= 32 when 1) and
+ *   k_blocks (> 0) without a GPU, and writes the cubin's path into path_out
+ *   (path_len bytes, NUL-terminated; may be NULL).  Returns FG_OK,
+ *   FG_ERR_INVALID_ARG, FG_ERR_UNSUPPORTED (no NVRTC or sources) or
+ *   FG_ERR_CUDA (compilation failed; FG_JIT_VERBOSE=1 prints the log).
+ * fg_jit_stats: specialisations compiled / read from the disk cache by this
+ *   process so far, and GEMM launches that ran a runtime-compiled kernel (any
+ *   pointer may be NULL).
+ */
+FG8_API fg_status fg_jit_compile(int block_n, int pair, int k_blocks, char* path_out, size_t path_len);
+FG8_API void fg_jit_stats(int* compiled, int* loaded_from_disk, int* launches);
+
+/*
  * Few-rows normal GEMM that allocates nothing.  The pages have no counterpart
  * to this entry point: it is an addition of this library.
  *

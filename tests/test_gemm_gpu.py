@@ -156,18 +156,60 @@ def test_repeated_launches_on_a_side_stream(fg):
     check(outs[0].double().cpu().numpy(), ref)
 
 
-def test_num_sms_limit_keeps_results(fg):
+@pytest.mark.parametrize("pair,bn,sms,M,N,K", [(0, 128, 8, 640, 640, 2048), (0, 128, 7, 640, 640, 2048),
+                                               (0, 256, 9, 1024, 1280, 3072), (1, 256, 12, 1024, 1280, 3072),
+                                               (1, 128, 12, 768, 640, 1536), (0, 64, 5, 384, 448, 1024)])
+def test_stream_k_split_tiles_match_oracle(fg, monkeypatch, pair, bn, sms, M, N, K):
+    """With the SM budget chosen so that the last wave of tiles is poorly
+    filled, the tile kernel processes the first waves whole and splits the
+    (tile, K block) iterations of the rest over the CTAs: pieces that end
+    inside a tile publish FP32 partial sums, the piece that finishes a tile
+    adds them in a fixed order.  Every element is checked against the oracle,
+    and two launches must agree bit for bit."""
+    monkeypatch.setenv("FG_FORCE_BLOCK_N", str(bn))
+    monkeypatch.setenv("FG_FORCE_PAIR", str(pair))
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(0, 80) + bn + sms)
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    full = fg.get_num_sms()
+    try:
+        fg.set_num_sms(sms)
+        D1 = fg.fp8_gemm_nt(A, sfa, B, sfb)
+        D2 = fg.fp8_gemm_nt(A, sfa, B, sfb)
+        monkeypatch.setenv("FG_STREAMK", "0")
+        D3 = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    finally:
+        fg.set_num_sms(full)
+    torch.cuda.synchronize()
+    assert torch.equal(D1, D2)
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    check(D1.double().cpu().numpy(), ref)
+    check(D3.double().cpu().numpy(), ref)
+
+
+def test_num_sms_limit_keeps_results(fg, monkeypatch):
+    """An SM budget changes only the schedule.  Without K splitting every
+    output sums its K blocks in order, so the bits do not change; with 7 SMs
+    the 16 tiles leave a ragged last wave that stream-K splits, which regroups
+    the FP32 sums (still deterministic, and within tolerance of the oracle)."""
     x = synth.normal_inputs(512, 1024, 512, seed=synth.seed_for(0, 71))
     A, sfa, B, sfb = to_gpu_normal(fg, x)
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
     full = fg.get_num_sms()
     D0 = fg.fp8_gemm_nt(A, sfa, B, sfb)
     try:
         fg.set_num_sms(7)
         assert fg.get_num_sms() == 7
         D1 = fg.fp8_gemm_nt(A, sfa, B, sfb)
+        D2 = fg.fp8_gemm_nt(A, sfa, B, sfb)
+        monkeypatch.setenv("FG_STREAMK", "0")
+        D3 = fg.fp8_gemm_nt(A, sfa, B, sfb)
     finally:
         fg.set_num_sms(full)
-    assert torch.equal(D0, D1)
+    torch.cuda.synchronize()
+    assert torch.equal(D1, D2)
+    assert torch.equal(D0, D3)
+    check(D1.double().cpu().numpy(), ref)
+    check(D0.double().cpu().numpy(), ref)
 
 
 # ----------------------------------------------------------- grouped GEMMs --

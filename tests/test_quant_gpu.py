@@ -57,6 +57,39 @@ def test_quantiser_special_blocks(fg):
     run_and_compare(fg, x)
 
 
+def e4m3_positive_values():
+    """Every finite positive E4M3 value, from the format's definition (bias
+    7, subnormals m/8 * 2^-6), in increasing order."""
+    vals = [m / 8.0 * 2.0 ** -6 for m in range(1, 8)]
+    vals += [(1 + m / 8.0) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8) if not (e == 15 and m == 7)]
+    return np.array(sorted(vals))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantiser_rounding_boundaries(fg, dtype):
+    """Quotients x / scale within a few FP32 units in the last place of every
+    rounding boundary of E4M3 (the midpoint between two neighbouring codes),
+    on both sides and at the boundary itself, for blocks with many different
+    scales: the codes must equal the oracle's, which divides in IEEE FP32."""
+    rng = np.random.default_rng(11)
+    vals = e4m3_positive_values()
+    mids = (vals[:-1] + vals[1:]) / 2.0
+    mids = np.concatenate([[vals[0] / 2.0], mids])          # the boundary between 0 and the smallest code
+    offs = np.array([-3, -2, -1, 0, 1, 2, 3], dtype=np.float64) * 2.0 ** -23
+    targets = (mids[:, None] * (1.0 + offs[None, :])).reshape(-1)
+    rows = []
+    for _ in range(64):
+        amax = np.float32(np.exp(rng.uniform(np.log(1e-3), np.log(1e3))))
+        scale = np.float32(max(amax, np.float32(1e-4))) / np.float32(448.0)
+        t = rng.choice(targets, 127)
+        sign = rng.choice([-1.0, 1.0], 127)
+        body = (sign * t).astype(np.float64) * np.float64(scale)
+        block = np.concatenate([[amax], np.clip(body, -amax, amax)]).astype(np.float32)
+        rows.append(block[rng.permutation(128)])
+    x = torch.from_numpy(np.stack(rows).reshape(8, 8 * 128))
+    run_and_compare(fg, x.to(dtype))
+
+
 def test_quantised_activations_feed_the_gemm(fg):
     """Quantising on the GPU and then multiplying gives the GEMM of the
     oracle's own quantisation of the same activations."""
