@@ -210,6 +210,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::tmem_alloc(tmem_slot, S::TMEM_COLS);
         ptx::tmem_relinquish();
     }
+    // Global memory is read or written only after the grids this launch
+    // depends on are done (programmatic dependent launch).
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();

@@ -271,8 +271,12 @@ Choice choose_config(int layout, int rows, int groups, int valid_rows, int N, in
     const char* force_pair = std::getenv("FG_FORCE_PAIR");
     const int fbn = force ? std::atoi(force) : 0;
     const int fpair = force_pair ? std::atoi(force_pair) : -1;
-    // CTA pairs halve each SM's B loads; FG_FORCE_PAIR=0/1 forbids/forces them.
-    const bool pair_ok = fpair != 0 && num_sms >= 2 && !(layout == LAYOUT_CONTIGUOUS && rows / BM > MAX_PAIR_LIST);
+    // CTA pairs halve each SM's B loads.  Measured on B200 they win a few per
+    // cent on the normal layout, tie on contiguous groups and lose on masked
+    // groups (whose 256-row tiles compute rows past masked_m), so by default
+    // only the normal layout considers them; FG_FORCE_PAIR=0/1 forbids/forces.
+    const bool pair_ok = num_sms >= 2 && !(layout == LAYOUT_CONTIGUOUS && rows / BM > MAX_PAIR_LIST) &&
+                         (fpair == 1 || (fpair != 0 && layout == LAYOUT_NORMAL));
     double best_t = 1e300;
     for (int pair = 0; pair <= 1; ++pair) {
         if (pair && !pair_ok) continue;

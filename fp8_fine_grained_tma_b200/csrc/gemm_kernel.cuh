@@ -459,6 +459,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::tmem_relinquish();
         }
     }
+    // Everything above touched only this CTA's own memory; global memory is
+    // read or written only after the grids this launch depends on are done.
+    ptx::griddep_wait();
+    ptx::griddep_launch_dependents();
     if (PAIR && p.layout == LAYOUT_CONTIGUOUS && warp == 0) {
         // The stage ring is free until the roles start: use it for the tags.
         const int n = build_pair_list(p, reinterpret_cast<int*>(stage_base), pair_list);
@@ -546,9 +550,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             while (w == 0 && sch.get(p, t)) {
                 for (int kb = t.kb0; kb < t.kb1; ++kb, ++g) {
                     if (g % NUM_MMA_WARPS == j) {
-                        w = wait_bar(&tempty[buf], bphase ^ 1u, limit, abort_flag);
-                        if (w) break;
+                        // The stage is normally loaded long before the accumulator
+                        // is released: wait for it first, so that nothing but the
+                        // fence stands between the release and the first MMA.
                         w = wait_bar(&full[stage], phase, limit, abort_flag);
+                        if (w) break;
+                        w = wait_bar(&tempty[buf], bphase ^ 1u, limit, abort_flag);
                         if (w) break;
                         ptx::tc_fence_after();
                         const uint32_t a_addr =

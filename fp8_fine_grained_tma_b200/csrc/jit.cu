@@ -341,14 +341,20 @@ fg_status jit_launch_gemm(int bn, bool pair, const CUtensorMap& ta, const CUtens
     cfg.blockDimZ = 1;
     cfg.sharedMemBytes = static_cast<unsigned>(smem);
     cfg.hStream = reinterpret_cast<CUstream>(stream);
-    CUlaunchAttribute attr[1];
+    CUlaunchAttribute attr[2];
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    if (pdl_enabled()) {
+        attr[cfg.numAttrs].id = CU_LAUNCH_ATTRIBUTE_PROGRAMMATIC_STREAM_SERIALIZATION;
+        attr[cfg.numAttrs].value.programmaticStreamSerializationAllowed = 1;
+        ++cfg.numAttrs;
+    }
     if (pair) {
-        attr[0].id = CU_LAUNCH_ATTRIBUTE_CLUSTER_DIMENSION;
-        attr[0].value.clusterDim.x = 2;
-        attr[0].value.clusterDim.y = 1;
-        attr[0].value.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[cfg.numAttrs].id = CU_LAUNCH_ATTRIBUTE_CLUSTER_DIMENSION;
+        attr[cfg.numAttrs].value.clusterDim.x = 2;
+        attr[cfg.numAttrs].value.clusterDim.y = 1;
+        attr[cfg.numAttrs].value.clusterDim.z = 1;
+        ++cfg.numAttrs;
     }
     CUtensorMap a = ta, b = tb, d = td;
     GemmParams pp = p;

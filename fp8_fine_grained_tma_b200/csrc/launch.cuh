@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cstdlib>
 
 #include "gemm_kernel.cuh"
 
@@ -16,6 +17,15 @@ constexpr int kMaxDynamicSmem = 232448;
 // schedulers), reserved out of kMaxDynamicSmem when the stages are sized.
 constexpr int kGemmStaticSmem = 1024;
 static_assert(NUM_EPI_WARPS * sizeof(TileScheduler<true>) <= kGemmStaticSmem, "static shared memory");
+
+// Programmatic dependent launch: a GEMM launched right after another kernel
+// in the same stream may start its prologue (barrier set-up, TMEM allocation)
+// while that kernel finishes; the kernels wait (griddepcontrol.wait) before
+// touching global memory.  FG_PDL=0 turns it off.
+inline bool pdl_enabled() {
+    const char* env = std::getenv("FG_PDL");
+    return !(env && std::atoi(env) == 0);
+}
 
 // Launches fg8_gemm_kernel<BN, PAIR> on `grid` CTAs (PAIR: clusters of two).
 // On first use per device it checks the build's register count (the in-kernel
@@ -51,14 +61,20 @@ cudaError_t launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, con
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem_bytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    if (pdl_enabled()) {
+        attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+        ++cfg.numAttrs;
+    }
     if (PAIR) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+        attr[cfg.numAttrs].val.clusterDim.x = 2;
+        attr[cfg.numAttrs].val.clusterDim.y = 1;
+        attr[cfg.numAttrs].val.clusterDim.z = 1;
+        ++cfg.numAttrs;
         // A persistent grid must fit on the device at once: clusters that do not
         // would start only after others finish.  Query (once per device, at the
         // largest shared-memory size, which all launches stay within) how many
@@ -66,6 +82,8 @@ cudaError_t launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, con
         int mc = max_clusters[dev & 63].load();
         if (mc == 0) {
             cudaLaunchConfig_t q = cfg;
+            q.attrs = &attr[cfg.numAttrs - 1];   // the cluster dimension only
+            q.numAttrs = 1;
             q.dynamicSmemBytes = kMaxDynamicSmem - kGemmStaticSmem;
             e = cudaOccupancyMaxActiveClusters(&mc, kernel, &q);
             if (e != cudaSuccess) return e;

@@ -129,6 +129,13 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 }
 
 // Bring the line holding `p` into L1 (no register, no completion to wait for).
+// Programmatic dependent launch: wait until the grids this one depends on
+// have completed and their memory is visible (a no-op when the launch had no
+// programmatic dependency), and let the next grid in the stream start its
+// prologue early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_l1(const void* p) {
     asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }

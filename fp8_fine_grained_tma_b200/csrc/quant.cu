@@ -28,7 +28,10 @@ namespace fg8q {
 
 constexpr int QBLK = 128;
 constexpr int QTHREADS = 256;
-constexpr int QUNROLL = 2;   // blocks per warp whose loads are in flight together
+// Blocks per warp whose loads are in flight together: 1 KiB per warp for
+// either input type, enough bytes in flight per SM to cover HBM latency.
+template <typename T>
+__host__ __device__ constexpr int qunroll() { return sizeof(T) == 2 ? 4 : 2; }
 
 __device__ __forceinline__ float4 load4(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
 
@@ -79,6 +82,7 @@ __global__ void __launch_bounds__(QTHREADS, 8) quantize_kernel(const T* __restri
     const int lane = threadIdx.x % 32;
     const long long warps = static_cast<long long>(gridDim.x) * (QTHREADS / 32);
     const long long w0 = static_cast<long long>(blockIdx.x) * (QTHREADS / 32) + threadIdx.x / 32;
+    constexpr int QUNROLL = qunroll<T>();
     for (long long base = w0; base < nblk; base += warps * QUNROLL) {
         float4 v[QUNROLL];
 #pragma unroll
@@ -150,7 +154,8 @@ extern "C" fg_status fg_quantize_fp8_activations(const void* x, int x_is_bf16, v
     if (sms <= 0) return FG_ERR_NO_DEVICE;
     const int m_pad = (M + 3) / 4 * 4;
     const long long nblk = static_cast<long long>(M) * (K / QBLK);
-    const long long warps_needed = (nblk + QUNROLL - 1) / QUNROLL;
+    const int unroll = x_is_bf16 ? qunroll<__nv_bfloat16>() : qunroll<float>();
+    const long long warps_needed = (nblk + unroll - 1) / unroll;
     const long long blocks_needed = (warps_needed + QTHREADS / 32 - 1) / (QTHREADS / 32);
     const int grid = static_cast<int>(blocks_needed < 8LL * sms ? (blocks_needed > 0 ? blocks_needed : 1) : 8LL * sms);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

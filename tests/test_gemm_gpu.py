@@ -186,11 +186,16 @@ def test_stream_k_split_tiles_match_oracle(fg, monkeypatch, pair, bn, sms, M, N,
     check(D3.double().cpu().numpy(), ref)
 
 
-def test_num_sms_limit_keeps_results(fg, monkeypatch):
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_num_sms_limit_keeps_results(fg, pair, monkeypatch):
     """An SM budget changes only the schedule.  Without K splitting every
     output sums its K blocks in order, so the bits do not change; with 7 SMs
-    the 16 tiles leave a ragged last wave that stream-K splits, which regroups
-    the FP32 sums (still deterministic, and within tolerance of the oracle)."""
+    the ragged last wave is split by stream-K, which regroups the FP32 sums
+    (still deterministic, and within tolerance of the oracle).  The tile shape
+    is fixed: tiles of another width or CTA pairing may round differently
+    inside the tensor core."""
+    monkeypatch.setenv("FG_FORCE_BLOCK_N", "128")
+    monkeypatch.setenv("FG_FORCE_PAIR", pair)
     x = synth.normal_inputs(512, 1024, 512, seed=synth.seed_for(0, 71))
     A, sfa, B, sfb = to_gpu_normal(fg, x)
     ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
