@@ -187,6 +187,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint64_t limit = p.wait_limit_ns;
     const uint64_t drain_limit = 2000000000ull;
 
+    // The producer's walk over this CTA's (unit, K block) sequence.  Its first
+    // p.stages loads need no free stage, so the producer issues them right
+    // after initialising the barriers, before the TMEM allocation and the
+    // block-wide barrier: the first bytes are on their way during the set-up.
+    DecodeCursor pcur(p, blockIdx.x, gridDim.x);
+    int preloaded = 0;
     if (warp == PRODUCER_WARP && lane == 0) {
         for (int s = 0; s < p.stages; ++s) {
             ptx::mbar_init(&full[s], 1);
@@ -205,6 +211,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::fence_mbarrier_init();
         ptx::prefetch_tensormap(&tmA);
         ptx::prefetch_tensormap(&tmB);
+        ptx::griddep_wait();
+        for (; pcur.valid && preloaded < p.stages; ++preloaded, pcur.advance(p, gridDim.x)) {
+            uint8_t* sb = stage_base + static_cast<size_t>(preloaded) * S::STAGE_BYTES;
+            ptx::mbar_arrive_expect_tx(&full[preloaded], S::STAGE_BYTES);
+            ptx::tma_load_3d(sb, &tmB, &full[preloaded], pcur.kb * BK, pcur.d.tile * BM, 0);
+            ptx::tma_load_3d(sb + S::B_BYTES, &tmA, &full[preloaded], pcur.kb * BK, 0, 0);
+        }
     }
     if (warp == MMA_WARP) {
         ptx::tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -223,24 +236,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::setmaxnreg_dec<DEC_REGS_PRODUCER>();
         if (warp == PRODUCER_WARP) {
             if (lane == 0) {
-                int stage = 0;
-                uint32_t phase = 0;
-                int issued = 0;
+                // Continue after the loads issued during the set-up.
+                int stage = preloaded == p.stages ? 0 : preloaded;
+                uint32_t phase = preloaded == p.stages ? 1u : 0u;
+                int issued = preloaded;
                 int w = 0;
-                DecodeUnit d;
-                for (int u = blockIdx.x; w == 0 && decode_unit(p, u, d); u += gridDim.x) {
-                    for (int kb = d.kb0; kb < d.kb1; ++kb) {
-                        w = wait_bar(&empty[stage], phase ^ 1u, limit, abort_flag);
-                        if (w) break;
-                        uint8_t* sb = stage_base + static_cast<size_t>(stage) * S::STAGE_BYTES;
-                        ptx::mbar_arrive_expect_tx(&full[stage], S::STAGE_BYTES);
-                        ptx::tma_load_3d(sb, &tmB, &full[stage], kb * BK, d.tile * BM, 0);
-                        ptx::tma_load_3d(sb + S::B_BYTES, &tmA, &full[stage], kb * BK, 0, 0);
-                        ++issued;
-                        if (++stage == p.stages) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
+                for (; w == 0 && pcur.valid; pcur.advance(p, gridDim.x)) {
+                    w = wait_bar(&empty[stage], phase ^ 1u, limit, abort_flag);
+                    if (w) break;
+                    uint8_t* sb = stage_base + static_cast<size_t>(stage) * S::STAGE_BYTES;
+                    ptx::mbar_arrive_expect_tx(&full[stage], S::STAGE_BYTES);
+                    ptx::tma_load_3d(sb, &tmB, &full[stage], pcur.kb * BK, pcur.d.tile * BM, 0);
+                    ptx::tma_load_3d(sb + S::B_BYTES, &tmA, &full[stage], pcur.kb * BK, 0, 0);
+                    ++issued;
+                    if (++stage == p.stages) {
+                        stage = 0;
+                        phase ^= 1u;
                     }
                 }
                 if (w == 2) record_error(p.status, ERR_TIMEOUT, ROLE_PRODUCER);
@@ -269,9 +280,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int u = blockIdx.x; w == 0 && decode_unit(p, u, d); u += gridDim.x) {
                     for (int kb = d.kb0; kb < d.kb1; ++kb, ++g) {
                         if (g % NUM_MMA_WARPS == j) {
-                            w = wait_bar(&tempty[buf], bphase ^ 1u, limit, abort_flag);
-                            if (w) break;
                             w = wait_bar(&full[stage], phase, limit, abort_flag);
+                            if (w) break;
+                            w = wait_bar(&tempty[buf], bphase ^ 1u, limit, abort_flag);
                             if (w) break;
                             ptx::tc_fence_after();
                             const uint32_t b_addr =
