@@ -13,10 +13,11 @@
 // so the block's largest magnitude lands on 448.  The 1e-4 floor keeps an
 // all-zero block finite.
 //
-// B200 design: the op is HBM-bound (5 bytes per FP32 element, 3 per BF16), so
-// one warp handles one 128-element block with 16-byte (FP32) or 8-byte (BF16)
-// coalesced loads, a 5-step shuffle max, and one 4-byte store of four codes
-// per lane; each warp walks several blocks with their loads issued together.
+// B200 design: the op should be HBM-bound (5 bytes per FP32 element, 3 per
+// BF16), so the per-element work is kept to a few instructions: eight lanes
+// share a 128-element block (16 elements each, 16-byte coalesced loads, a
+// 3-step shuffle max, one 16-byte store of codes per lane) and a warp covers
+// four consecutive blocks per instruction.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -28,21 +29,41 @@ namespace fg8q {
 
 constexpr int QBLK = 128;
 constexpr int QTHREADS = 256;
-// Blocks per warp whose loads are in flight together: 1 KiB per warp for
-// either input type, enough bytes in flight per SM to cover HBM latency.
-template <typename T>
-__host__ __device__ constexpr int qunroll() { return sizeof(T) == 2 ? 4 : 2; }
+// Eight lanes quantise one 128-element block (16 elements each), so a warp
+// instruction serves four blocks: the per-block work (the amax reduction, the
+// scale, its reciprocal and the scale store) is shared four ways instead of
+// being paid once per 4 elements.  Latency is hidden by occupancy: 48 warps
+// per SM (six CTAs of 256 threads, at most 40 registers each), each with one
+// group of four blocks in flight, measured faster than fewer warps with two
+// groups each or with the next group prefetched.
+constexpr int QLANES = 8;
+constexpr int QEL = QBLK / QLANES;          // 16 elements per lane
+constexpr int QU = 1;
+constexpr int QMIN_BLOCKS = 6;
 
-__device__ __forceinline__ float4 load4(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+// 16 consecutive elements as FP32 (streaming loads: the input is read once).
+__device__ __forceinline__ void load16(const float* p, float (&v)[QEL]) {
+#pragma unroll
+    for (int i = 0; i < QEL / 4; ++i) {
+        const float4 f = __ldcs(reinterpret_cast<const float4*>(p) + i);
+        v[4 * i] = f.x;
+        v[4 * i + 1] = f.y;
+        v[4 * i + 2] = f.z;
+        v[4 * i + 3] = f.w;
+    }
+}
 
-__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
-    const uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));
-    float4 f;
-    f.x = __uint_as_float(u.x << 16);
-    f.y = __uint_as_float(u.x & 0xFFFF0000u);
-    f.z = __uint_as_float(u.y << 16);
-    f.w = __uint_as_float(u.y & 0xFFFF0000u);
-    return f;
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[QEL]) {
+#pragma unroll
+    for (int i = 0; i < QEL / 8; ++i) {
+        const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p) + i);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
 }
 
 // x / b rounded to nearest even, given y = the correctly rounded reciprocal
@@ -51,19 +72,25 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
 // rounded once is the correctly rounded quotient when q is within one unit in
 // the last place of x / b.  x * y alone can be 1.5 units off, so one residual
 // step brings it within one unit and a second gives the correctly rounded
-// result.  Computed on |x| with the sign put back at the end, so that -0 / b
-// stays -0 (a residual step would turn it into +0).  Used for the per-element
-// quotients; valid for the normal scales and |x / b| <= 448 (plus rounding)
-// of the quantiser.  The tests check the codes bit for bit against IEEE
-// division on values within a few units of every E4M3 rounding boundary.
-__device__ __forceinline__ float div_rn(float x, float b, float y) {
-    const float a = fabsf(x);
-    float q = a * y;
-    float r = fmaf(-q, b, a);
-    q = fmaf(r, y, q);
-    r = fmaf(-q, b, a);
-    q = fmaf(r, y, q);
-    return copysignf(q, x);
+// result.  The sign of x is put back at the end, so that -0 / b stays -0 (a
+// residual step would turn it into +0).  Used for the per-element quotients;
+// valid for the normal scales and |x / b| <= 448 (plus rounding) of the
+// quantiser.  The tests check the codes bit for bit against IEEE division on
+// values within a few units of every E4M3 rounding boundary.
+__device__ __forceinline__ float2 div_rn2(float2 x, float b, float y) {
+    // Two quotients per instruction (packed FP32 multiply and FMA, each half
+    // rounded to nearest as the scalar operation would be).  The steps run on
+    // the signed values: round-to-nearest-even is symmetric, so the result is
+    // exactly the negated quotient of |x| except for a zero, whose sign the
+    // final copysign restores.
+    const float2 y2 = make_float2(y, y);
+    const float2 nb2 = make_float2(-b, -b);
+    float2 q = __fmul2_rn(x, y2);
+    float2 r = __ffma2_rn(q, nb2, x);
+    q = __ffma2_rn(r, y2, q);
+    r = __ffma2_rn(q, nb2, x);
+    q = __ffma2_rn(r, y2, q);
+    return make_float2(copysignf(q.x, x.x), copysignf(q.y, x.y));
 }
 
 // Four FP32 -> four E4M3 codes (round to nearest even, saturating), byte i = value i.
@@ -75,35 +102,53 @@ __device__ __forceinline__ uint32_t to_e4m3x4(float a, float b, float c, float d
 }
 
 template <typename T>
-__global__ void __launch_bounds__(QTHREADS, 8) quantize_kernel(const T* __restrict__ x, uint8_t* __restrict__ q,
+__global__ void __launch_bounds__(QTHREADS, QMIN_BLOCKS) quantize_kernel(const T* __restrict__ x, uint8_t* __restrict__ q,
                                                             float* __restrict__ sfa, int M, int K, int m_pad) {
     const int KB = K / QBLK;
     const long long nblk = static_cast<long long>(M) * KB;
     const int lane = threadIdx.x % 32;
+    const int sub = lane / QLANES;                  // block of the warp's group of four
+    const int l8 = lane % QLANES;                   // 16-element slice of that block
     const long long warps = static_cast<long long>(gridDim.x) * (QTHREADS / 32);
     const long long w0 = static_cast<long long>(blockIdx.x) * (QTHREADS / 32) + threadIdx.x / 32;
-    constexpr int QUNROLL = qunroll<T>();
-    for (long long base = w0; base < nblk; base += warps * QUNROLL) {
-        float4 v[QUNROLL];
+    const long long step = warps * 4;               // blocks per sweep of the whole grid
+    for (long long base = w0 * 4; base < nblk; base += step * QU) {
+        float v[QU][QEL];
 #pragma unroll
-        for (int u = 0; u < QUNROLL; ++u) {
-            const long long b = base + u * warps;
-            v[u] = b < nblk ? load4(x + b * QBLK + lane * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < QU; ++u) {
+            const long long b = base + u * step + sub;
+            if (b < nblk) {
+                load16(x + b * QBLK + l8 * QEL, v[u]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < QEL; ++i) v[u][i] = 0.0f;
+            }
         }
 #pragma unroll
-        for (int u = 0; u < QUNROLL; ++u) {
-            const long long b = base + u * warps;
-            float amax = fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w)));
+        for (int u = 0; u < QU; ++u) {
+            const long long b = base + u * step + sub;
+            float amax = 0.0f;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            if (b >= nblk) continue;   // warp-uniform
+            for (int i = 0; i < QEL; ++i) amax = fmaxf(amax, fabsf(v[u][i]));
+#pragma unroll
+            for (int o = QLANES / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            if (b >= nblk) continue;
             const float scale = fmaxf(amax, 1e-4f) / 448.0f;
             const float rcp = __frcp_rn(scale);
-            const uint32_t codes = to_e4m3x4(div_rn(v[u].x, scale, rcp), div_rn(v[u].y, scale, rcp),
-                                             div_rn(v[u].z, scale, rcp), div_rn(v[u].w, scale, rcp));
-            __stcs(reinterpret_cast<uint32_t*>(q + b * QBLK) + lane, codes);
-            if (lane == 0) {
-                const long long m = b / KB;
+            uint32_t c[QEL / 4];
+#pragma unroll
+            for (int i = 0; i < QEL / 4; ++i) {
+                const float2 lo = div_rn2(make_float2(v[u][4 * i], v[u][4 * i + 1]), scale, rcp);
+                const float2 hi = div_rn2(make_float2(v[u][4 * i + 2], v[u][4 * i + 3]), scale, rcp);
+                c[i] = to_e4m3x4(lo.x, lo.y, hi.x, hi.y);
+            }
+            __stcs(reinterpret_cast<uint4*>(q + b * QBLK + l8 * QEL), make_uint4(c[0], c[1], c[2], c[3]));
+            if (l8 == 0) {
+                // Block b is row m, K block kb (32-bit division whenever the
+                // block count allows it).
+                long long m;
+                if (nblk <= 0x7fffffffLL) m = static_cast<long long>(static_cast<unsigned>(b) / static_cast<unsigned>(KB));
+                else m = b / KB;
                 const int kb = static_cast<int>(b - m * KB);
                 sfa[static_cast<long long>(kb) * m_pad + m] = scale;
             }
@@ -154,10 +199,10 @@ extern "C" fg_status fg_quantize_fp8_activations(const void* x, int x_is_bf16, v
     if (sms <= 0) return FG_ERR_NO_DEVICE;
     const int m_pad = (M + 3) / 4 * 4;
     const long long nblk = static_cast<long long>(M) * (K / QBLK);
-    const int unroll = x_is_bf16 ? qunroll<__nv_bfloat16>() : qunroll<float>();
-    const long long warps_needed = (nblk + unroll - 1) / unroll;
+    const long long warps_needed = (nblk + 4 * QU - 1) / (4 * QU);
     const long long blocks_needed = (warps_needed + QTHREADS / 32 - 1) / (QTHREADS / 32);
-    const int grid = static_cast<int>(blocks_needed < 8LL * sms ? (blocks_needed > 0 ? blocks_needed : 1) : 8LL * sms);
+    const int grid = static_cast<int>(blocks_needed < static_cast<long long>(QMIN_BLOCKS) * sms ? (blocks_needed > 0 ? blocks_needed : 1)
+                                                                          : static_cast<long long>(QMIN_BLOCKS) * sms);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (x_is_bf16)
         quantize_kernel<__nv_bfloat16><<<grid, QTHREADS, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
