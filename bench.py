@@ -103,6 +103,7 @@ class Case:
         self.plan = None          # launch plan (fg.query_plan)
         self.copies = copies
         self.config = None        # workload (configuration) the GEMM belongs to
+        self.decode_sized = False  # few rows of A: also timed back to back
 
 
 def n_copies(footprint_bytes):
@@ -148,6 +149,7 @@ def build_cases(fg, synth, wl, device):
 
                 c = Case(f"M{M}_N{N}_K{K}", flops, hbm, run, host={"x": x, "D": D}, copies=len(sets))
                 c.plan = fg.query_plan("normal", M, N, K)
+                c.decode_sized = M <= 256
                 cases.append(c)
     elif kind == "contiguous":
         for si, (N, K) in enumerate(wl["shapes"]):
@@ -454,7 +456,7 @@ def main(argv=None):
     per_case_ms = [sum(evs[s][ci][0].elapsed_time(evs[s][ci][1]) for s in range(args.steps))
                    for ci in range(len(cases))]
 
-    # Decode-kernel GEMMs also run as a decode step runs its layers: launches
+    # Decode-sized GEMMs (M <= 256) also run as a decode step runs its layers: launches
     # back to back on the stream, each on the next operand copy (the copies
     # total more than twice L2), so programmatic dependent launch overlaps each
     # kernel's set-up with the previous one's tail.  Per-launch time = chain
@@ -462,7 +464,7 @@ def main(argv=None):
     # not use it.
     chain_us = {}
     for ci, c in enumerate(cases):
-        if args.no_chain or not (c.plan and c.plan.get("kernel") == "decode"):
+        if args.no_chain or not c.decode_sized:
             continue
         n = max(8, c.copies)
         for i in range(n):

@@ -20,7 +20,10 @@
 
 namespace fg8 {
 
-#define FG8_DECLARE_BOTH(BN) FG8_DECLARE_LAUNCH_ONE(BN, false) FG8_DECLARE_LAUNCH_ONE(BN, true)
+#define FG8_DECLARE_BOTH(BN)                                 \
+    FG8_DECLARE_LAUNCH_ONE(BN, false) FG8_DECLARE_LAUNCH_ONE(BN, true) \
+    template <>                                              \
+    cudaError_t gemm_max_split_clusters<BN>(int cluster, int* out);
 FG8_FOR_EACH_BN(FG8_DECLARE_BOTH)
 #undef FG8_DECLARE_BOTH
 FG8_FOR_EACH_MT(FG8_DECLARE_DECODE_LAUNCH)
@@ -309,22 +312,22 @@ int choose_stages(int bn, bool pair) {
 
 template <int BN>
 cudaError_t launch_either(bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                          const GemmParams& p, int grid, size_t smem, cudaStream_t st) {
+                          const GemmParams& p, int grid, size_t smem, cudaStream_t st, int cluster) {
     if constexpr (BN >= 32) {
-        if (pair) return launch_gemm<BN, true>(ta, tb, td, p, grid, smem, st);
+        if (pair) return launch_gemm<BN, true>(ta, tb, td, p, grid, smem, st, 2);
     } else {
         if (pair) return cudaErrorInvalidValue;
     }
-    return launch_gemm<BN, false>(ta, tb, td, p, grid, smem, st);
+    return launch_gemm<BN, false>(ta, tb, td, p, grid, smem, st, cluster);
 }
 
 fg_status launch_bn(int bn, bool pair, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                    const GemmParams& p, int grid, size_t smem, cudaStream_t st) {
+                    const GemmParams& p, int grid, size_t smem, cudaStream_t st, int cluster = 1) {
     cudaError_t e = cudaErrorInvalidValue;
     switch (bn) {
 #define FG8_CASE(BNV) \
     case BNV:         \
-        e = launch_either<BNV>(pair, ta, tb, td, p, grid, smem, st); \
+        e = launch_either<BNV>(pair, ta, tb, td, p, grid, smem, st, cluster); \
         break;
         FG8_FOR_EACH_BN(FG8_CASE)
 #undef FG8_CASE
@@ -619,6 +622,125 @@ fg_status get_streamk_workspace(int dev, cudaStream_t stream, size_t ws_bytes, s
     return FG_OK;
 }
 
+// ---- cluster split-K through the tile kernel (few rows) -----------------------
+// For M <= 128 the tile kernel covers all rows with one 128-row tile per column
+// block; its K blocks are split over the `ks` CTAs of a thread-block cluster,
+// which sum their FP32 partials through distributed shared memory.  With the
+// token rows on the MMA's M side each promotion thread scales one row by two
+// scalars per K block (the swap-AB decode kernel needs a scale per column).
+// FG_TILE_SPLITK=0 / 1 forbids / forces it; by default it serves 64 < M <= 128
+// when the splits stay long (see below).
+struct SplitKPlan {
+    bool on = false;
+    int bn = 0, ks = 0, ks_per = 0, tiles = 0;
+};
+
+cudaError_t max_split_clusters(int bn, int cluster, int* out) {
+    switch (bn) {
+#define FG8_CASE(BNV) \
+    case BNV:         \
+        return gemm_max_split_clusters<BNV>(cluster, out);
+        FG8_FOR_EACH_BN(FG8_CASE)
+#undef FG8_CASE
+        default:
+            return cudaErrorInvalidValue;
+    }
+}
+
+SplitKPlan splitk_plan(int M, int N, int K, int sms) {
+    SplitKPlan sp;
+    const char* env = std::getenv("FG_TILE_SPLITK");
+    const int mode = env ? std::atoi(env) : -1;
+    if (mode == 0 || M > BM) return sp;
+    if (mode < 0 && M <= 64) return sp;
+    const int KB = K / BK;
+    const int bn = N >= 256 ? 256 : (N + 15) / 16 * 16;
+    const int tiles = (N + bn - 1) / bn;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return sp;
+    }
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int>, int> cache;   // (device, bn, cluster) -> resident clusters
+    for (int ks = std::min({8, KB, sms / std::max(1, tiles)}); ks >= 2; --ks) {
+        const int ks_per = (KB + ks - 1) / ks;
+        const int ks2 = (KB + ks_per - 1) / ks_per;          // every split gets K blocks
+        if (ks2 < 2) continue;
+        int mc = 0;
+        {
+            std::lock_guard<std::mutex> lk(mu);
+            auto it = cache.find({dev, bn, ks2});
+            if (it != cache.end()) {
+                mc = it->second;
+            } else {
+                if (max_split_clusters(bn, ks2, &mc) != cudaSuccess) {
+                    cudaGetLastError();
+                    mc = 0;
+                }
+                cache[{dev, bn, ks2}] = mc;
+            }
+        }
+        if (tiles <= mc) {
+            // Measured on B200 (M=128, back-to-back launches): against the
+            // swap-AB decode kernel this wins only when each split still has
+            // many K blocks (7168 x 16384: 34 vs 49 us, 32 K blocks per split)
+            // and loses with short splits (7 to 10 K blocks: 17 to 20 vs 13 to
+            // 17 us), where its set-up and the cluster reduction dominate.
+            if (mode < 0 && ks_per < 24) return sp;
+            sp.on = true;
+            sp.bn = bn;
+            sp.ks = ks2;
+            sp.ks_per = ks_per;
+            sp.tiles = tiles;
+            return sp;
+        }
+    }
+    return sp;
+}
+
+fg_status run_gemm_splitk(const SplitKPlan& sp, const void* A, const float* sfa, const void* B, const float* sfb,
+                          void* D, int M, int N, int K, cudaStream_t stream) {
+    DeviceInfo* dev = nullptr;
+    fg_status st = current_device(&dev);
+    if (st != FG_OK) return st;
+    const int bn = sp.bn;
+    const int stages = choose_stages(bn, false);
+    const size_t smem = gemm_smem_bytes(stage_bytes_for(bn, false), stages, false);
+    // The partial of a split ([128 rows][bn] FP32) is staged in the stage ring.
+    if (static_cast<size_t>(BM) * bn * sizeof(float) > static_cast<size_t>(stages) * stage_bytes_for(bn, false))
+        return FG_ERR_UNSUPPORTED;
+    CUtensorMap ta, tb, td;
+    st = operand_map(A, K, M, 1, BM, &ta);
+    if (st != FG_OK) return st;
+    st = operand_map(B, K, N, 1, bn, &tb);
+    if (st != FG_OK) return st;
+    st = output_map(D, N, M, 1, &td);
+    if (st != FG_OK) return st;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.layout = LAYOUT_NORMAL;
+    p.rows = M;
+    p.N = N;
+    p.K = K;
+    p.G = 1;
+    p.KB = K / BK;
+    p.NB = (N + 127) / 128;
+    p.num_m_tiles = 1;
+    p.num_n_blocks = sp.tiles;
+    p.raster_m = 1;
+    p.stages = stages;
+    p.sfa_ld = static_cast<int>(fg_get_tma_aligned_size(M, 4));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.D = static_cast<__nv_bfloat16*>(D);
+    p.status = dev->status;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    p.ks = sp.ks;
+    p.ks_per = sp.ks_per;
+    return launch_bn(bn, false, ta, tb, td, p, sp.tiles * sp.ks, smem, stream, sp.ks);
+}
+
 // Shared by the three GEMM kinds once their arguments are checked.
 fg_status run_gemm(int layout, const void* A, const float* sfa, const void* B, const float* sfb, void* D,
                    const int* m_indices, const int* masked_m, int rows, int N, int K, int G, int valid_rows_hint,
@@ -750,8 +872,14 @@ fg_status fg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const f
     if (!aligned16(A) || !aligned16(B) || !aligned16(D) || !aligned16(sfa) || !aligned4(sfb))
         return FG_ERR_ALIGNMENT;
     if (static_cast<long long>(M) * N > kMaxDim * 4 || M > kMaxDim - 128) return FG_ERR_UNSUPPORTED;
-    if (M <= std::min(decode_max_rows(), 256))
+    if (M <= std::min(decode_max_rows(), 256)) {
+        DeviceInfo* dev = nullptr;
+        if (current_device(&dev) == FG_OK) {
+            const SplitKPlan sp = splitk_plan(M, N, K, effective_sms(*dev));
+            if (sp.on) return run_gemm_splitk(sp, A, sfa, B, sfb, D, M, N, K, reinterpret_cast<cudaStream_t>(stream));
+        }
         return run_decode(A, sfa, B, sfb, D, M, N, K, reinterpret_cast<cudaStream_t>(stream));
+    }
     return run_gemm(LAYOUT_NORMAL, A, sfa, B, sfb, D, nullptr, nullptr, M, N, K, 1, M,
                     reinterpret_cast<cudaStream_t>(stream));
 }
@@ -897,6 +1025,17 @@ fg_status fg_query_plan(int layout, int rows, int N, int K, int G, int expected_
         sms = g_num_sms.load();
     }
     if (layout == LAYOUT_NORMAL && rows <= std::min(decode_max_rows(), 256)) {
+        if (dev_id >= 0) {
+            const SplitKPlan sk = splitk_plan(rows, N, K, sms);
+            if (sk.on) {
+                *kernel_out = 0;
+                *tile_n_out = sk.bn;
+                *pair_out = 0;
+                *splits_out = sk.ks;
+                *cluster_out = sk.ks;
+                return FG_OK;
+            }
+        }
         const int mt = decode_tile_width(rows);
         const int stages = decode_stages(mt);
         const size_t smem = decode_smem_bytes(BM * BK + mt * BK, stages, mt);

@@ -7,6 +7,10 @@
 #endif
 
 namespace fg8 {
+template <>
+cudaError_t gemm_max_split_clusters<FG8_BN>(int cluster, int* out) {
+    return gemm_max_split_clusters_impl<FG8_BN>(cluster, out);
+}
 FG8_DEFINE_LAUNCH_ONE(FG8_BN, false)
 #if FG8_BN >= 32
 FG8_DEFINE_LAUNCH_ONE(FG8_BN, true)

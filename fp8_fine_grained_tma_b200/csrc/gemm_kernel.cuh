@@ -114,6 +114,12 @@ struct GemmParams {
     // CTA ([grid][NC][128][16]), sk_flags the epoch of the last partial each
     // promotion warp of each CTA published ([grid][8]); sk_epoch is this
     // launch's (never 0).
+    // Cluster split-K (normal layout, single CTAs, one row tile): CTA u of the
+    // grid handles tile u / ks, K blocks [s * ks_per, (s + 1) * ks_per) with
+    // s = u % ks; the ks CTAs of a tile form one thread-block cluster and sum
+    // their partials through distributed shared memory.  ks <= 1: off.
+    int ks;
+    int ks_per;
     int sk;                  // 1: stream-K on
     int sk_dp_tiles;         // tiles processed whole before the split ones
     long long sk_iters;      // (tiles - sk_dp_tiles) * KB
@@ -227,6 +233,20 @@ struct TileScheduler {
         t.kb0 = 0;
         t.kb1 = FG8_KB_CT > 0 ? FG8_KB_CT : p.KB;
         t.sk_first = -1;
+        if (!PAIR && p.ks > 1) {
+            // One (tile, K split) per CTA.
+            if (next >= p.num_m_tiles * p.num_n_blocks * p.ks) return false;
+            const int tile = next / p.ks;
+            const int split = next - tile * p.ks;
+            next += stride;
+            t.kb0 = split * p.ks_per;
+            t.kb1 = min(p.KB, t.kb0 + p.ks_per);
+            int m_tile;
+            raster(p, tile, m_tile, t.n_blk);
+            t.row0 = m_tile * BM;
+            t.g = 0;
+            return true;
+        }
         if (p.sk) {
             // Whole tiles first (unit, unit + units, ... below sk_dp_tiles), then
             // this unit's share of the split iterations, last piece first: a
@@ -805,6 +825,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 break;
             }
 
+            if (!PAIR && p.ks > 1) {
+                // Cluster split-K: stage this split's FP32 partial in the (now
+                // idle) stage ring as [chunk][row][16]; the cluster reduction
+                // after the role branches writes D.
+                float* part = reinterpret_cast<float*>(stage_base);
+#pragma unroll
+                for (int i = 0; i < CPW; ++i) {
+                    const int c = chunk0 + i;
+                    if (c >= NC) break;
+                    float4* dst = reinterpret_cast<float4*>(part + (static_cast<size_t>(c) * BM + row_in_tile) * 16);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_float4(acc[i][2 * q].x, acc[i][2 * q].y, acc[i][2 * q + 1].x, acc[i][2 * q + 1].y);
+                }
+                continue;
+            }
+
             // ---- stream-K: publish a partial sum, or add the earlier ones ----
             if (t.kb1 < p.KB) {
                 // This piece ends inside its tile: store its FP32 partial sum in
@@ -955,6 +992,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_before();
     __syncthreads();
     if constexpr (PAIR) ptx::cluster_sync();   // the leader's MMAs read the peer's shared memory until here
+    if (!PAIR && p.ks > 1) {
+        // Cluster split-K: once every split of the tile has staged its partial,
+        // CTA r of the cluster sums a slice of the tile's rows over all splits
+        // in split order (deterministic), reading the peers' shared memory, and
+        // writes them as BF16; the second barrier keeps each CTA's partial
+        // alive until its peers have read it.  Every thread takes both
+        // barriers, also after an abort.
+        ptx::cluster_sync();
+        if (warp < NUM_EPI_WARPS && !*abort_flag) {
+            const int S = p.ks;
+            const int r = static_cast<int>(ptx::cluster_ctarank());
+            int m_tile, n_blk;
+            TileScheduler<PAIR>::raster(p, static_cast<int>(blockIdx.x) / S, m_tile, n_blk);
+            const int row0 = m_tile * BM;
+            const int n0 = n_blk * BN;
+            const int rows = min(BM, p.rows - row0);
+            const int rs = (rows + S - 1) / S;
+            const int r0 = min(rows, r * rs);
+            const int r1 = min(rows, r0 + rs);
+            constexpr int Q = BN / 4;                         // 4-column groups of a row
+            const uint32_t base = ptx::smem_addr(stage_base);
+            for (int e = threadIdx.x; e < (r1 - r0) * Q; e += NUM_EPI_WARPS * 32) {
+                const int row = r0 + e / Q;
+                const int col = (e - (e / Q) * Q) * 4;
+                const int n = n0 + col;
+                if (n >= p.N) continue;                        // N % 16 == 0: the 4 columns are all in range
+                const uint32_t off =
+                    base + static_cast<uint32_t>((((col >> 4) * BM + row) * 16 + (col & 15)) * 4);
+                // All splits' loads in flight together, then the sum in split order.
+                float4 v[8];
+#pragma unroll
+                for (int sp = 0; sp < 8; ++sp)
+                    if (sp < S) v[sp] = ptx::ld_shared_cluster_v4(ptx::mapa_shared(off, static_cast<uint32_t>(sp)));
+                float4 sum = v[0];
+#pragma unroll
+                for (int sp = 1; sp < 8; ++sp) {
+                    if (sp < S) {
+                        sum.x += v[sp].x;
+                        sum.y += v[sp].y;
+                        sum.z += v[sp].z;
+                        sum.w += v[sp].w;
+                    }
+                }
+                uint2 pk;
+                pk.x = pack_bf16x2(sum.x, sum.y);
+                pk.y = pack_bf16x2(sum.z, sum.w);
+                *reinterpret_cast<uint2*>(p.D + static_cast<size_t>(row0 + row) * p.N + n) = pk;
+            }
+        }
+        ptx::cluster_sync();
+    }
     if (warp == MMA_WARP) {
         ptx::tc_fence_after();
         if constexpr (PAIR) ptx::tmem_dealloc_pair(tmem_base, S::TMEM_COLS);

@@ -27,17 +27,19 @@ inline bool pdl_enabled() {
     return !(env && std::atoi(env) == 0);
 }
 
-// Launches fg8_gemm_kernel<BN, PAIR> on `grid` CTAs (PAIR: clusters of two).
+// Launches fg8_gemm_kernel<BN, PAIR> on `grid` CTAs (PAIR: clusters of two;
+// otherwise clusters of `cluster` CTAs when cluster > 1, for the cluster
+// split-K mode, whose grid the host has checked to be resident at once).
 // On first use per device it checks the build's register count (the in-kernel
 // register split is safe only at exactly REGS_LAUNCH) and raises the kernel's
 // shared-memory limit.  Defined in gemm_inst.cu, one block width per object.
 template <int BN, bool PAIR>
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD, const GemmParams& p,
-                        int grid, size_t smem_bytes, cudaStream_t stream);
+                        int grid, size_t smem_bytes, cudaStream_t stream, int cluster);
 
 template <int BN, bool PAIR>
 cudaError_t launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
-                             const GemmParams& p, int grid, size_t smem_bytes, cudaStream_t stream) {
+                             const GemmParams& p, int grid, size_t smem_bytes, cudaStream_t stream, int cluster) {
     static std::atomic<unsigned long long> attr_set{0};
     static std::atomic<int> max_clusters[64];   // per device, 0 = not queried yet
     int dev = 0;
@@ -91,21 +93,60 @@ cudaError_t launch_gemm_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, con
             max_clusters[dev & 63].store(mc);
         }
         if (grid > 2 * mc) cfg.gridDim.x = static_cast<unsigned>(2 * mc);
+    } else if (cluster > 1) {
+        if (cluster > 8) return cudaErrorInvalidConfiguration;
+        attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+        attr[cfg.numAttrs].val.clusterDim.x = static_cast<unsigned>(cluster);
+        attr[cfg.numAttrs].val.clusterDim.y = 1;
+        attr[cfg.numAttrs].val.clusterDim.z = 1;
+        ++cfg.numAttrs;
+        // The host sized the grid from gemm_max_split_clusters (whole grid resident).
+        if (grid % cluster != 0) return cudaErrorInvalidConfiguration;
     }
     return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmD, p);
+}
+
+// Largest number of clusters of `cluster` single CTAs of fg8_gemm_kernel<BN,
+// false> that can be resident at once (cluster split-K sizing).
+template <int BN>
+cudaError_t gemm_max_split_clusters(int cluster, int* out);
+
+template <int BN>
+cudaError_t gemm_max_split_clusters_impl(int cluster, int* out) {
+    auto kernel = fg8_gemm_kernel<BN, false>;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMaxDynamicSmem - static_cast<int>(fa.sharedSizeBytes));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(cluster), 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = kMaxDynamicSmem - kGemmStaticSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaOccupancyMaxActiveClusters(out, kernel, &cfg);
 }
 
 #define FG8_DEFINE_LAUNCH_ONE(BN, PAIR)                                                                        \
     template <>                                                                                                \
     cudaError_t launch_gemm<BN, PAIR>(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,  \
-                                      const GemmParams& p, int grid, size_t smem_bytes, cudaStream_t stream) { \
-        return launch_gemm_impl<BN, PAIR>(tmA, tmB, tmD, p, grid, smem_bytes, stream);                         \
+                                      const GemmParams& p, int grid, size_t smem_bytes, cudaStream_t stream,   \
+                                      int cluster) {                                                           \
+        return launch_gemm_impl<BN, PAIR>(tmA, tmB, tmD, p, grid, smem_bytes, stream, cluster);                \
     }
 
 #define FG8_DECLARE_LAUNCH_ONE(BN, PAIR)                                                                       \
     template <>                                                                                                \
     cudaError_t launch_gemm<BN, PAIR>(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,  \
-                                      const GemmParams& p, int grid, size_t smem_bytes, cudaStream_t stream);
+                                      const GemmParams& p, int grid, size_t smem_bytes, cudaStream_t stream,   \
+                                      int cluster);
 
 // Block widths 16..256; CTA pairs from 32 (each CTA loads at least 16 B rows).
 #define FG8_FOR_EACH_BN(X) \

@@ -441,6 +441,7 @@ def test_decode_kernel_matches_oracle(fg, M, splits, reduce, monkeypatch):
     shared memory or through the global workspace; every token-tile width
     32..256.  Five splits of 8 K blocks leave the last split empty."""
     monkeypatch.setenv("FG_DECODE_MAX_M", "256")
+    monkeypatch.setenv("FG_TILE_SPLITK", "0")
     monkeypatch.setenv("FG_FORCE_SPLITS", splits)
     monkeypatch.setenv("FG_DECODE_CLUSTER", "0" if reduce == "workspace" else "1")
     N, K = 400, 1024
@@ -486,6 +487,7 @@ def test_decode_cluster_and_workspace_reductions_agree(fg, M, N, K, splits, monk
     """Both split-K reductions add the splits in the same order, so their
     results are equal element for element."""
     monkeypatch.setenv("FG_FORCE_SPLITS", splits)
+    monkeypatch.setenv("FG_TILE_SPLITK", "0")
     x = synth.normal_inputs(M, N, K, seed=synth.seed_for(4, 63) + M)
     A, sfa, B, sfb = to_gpu_normal(fg, x)
     monkeypatch.setenv("FG_DECODE_CLUSTER", "1")
@@ -497,6 +499,38 @@ def test_decode_cluster_and_workspace_reductions_agree(fg, M, N, K, splits, monk
     rows = sample_rows(M, 8, M)
     ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy(), rows=rows)
     check(D1[torch.from_numpy(rows).cuda()].double().cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 4096, 7168), (100, 2112, 7168), (96, 7168, 2048), (65, 400, 1536),
+                                   (1, 272, 1024), (17, 528, 640), (128, 256, 256), (128, 32768, 512)])
+def test_tile_split_k_matches_oracle(fg, M, N, K, monkeypatch):
+    """Few rows on the 128-row tile kernel with K split over the CTAs of a
+    cluster and the partials summed through distributed shared memory in split
+    order: every element against the oracle, ragged N and M, and the same
+    bits on a second launch."""
+    monkeypatch.setenv("FG_TILE_SPLITK", "1")
+    plan = fg.query_plan("normal", M, N, K)
+    tiles = -(-N // 256)
+    if plan["kernel"] != "tile":
+        pytest.skip(f"no resident cluster split for {tiles} tiles on this device: {plan}")
+    assert plan["splits"] >= 2 and plan["cluster"] == plan["splits"]
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(4, 70) + M + N)
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    D = torch.full((M, N), SENTINEL, dtype=torch.bfloat16, device="cuda")
+    fg.fp8_gemm_nt(A, sfa, B, sfb, D=D)
+    D2 = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    assert fg.get_last_device_status()[0] == 0
+    assert torch.equal(D, D2)
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    check(D.double().cpu().numpy(), ref)
+
+
+def test_tile_split_k_is_the_default_for_long_k_between_64_and_128_rows(fg, monkeypatch):
+    monkeypatch.delenv("FG_TILE_SPLITK", raising=False)
+    assert fg.query_plan("normal", 128, 7168, 16384)["kernel"] == "tile"
+    assert fg.query_plan("normal", 64, 7168, 16384)["kernel"] == "decode"
+    assert fg.query_plan("normal", 128, 2112, 7168)["kernel"] == "decode"
 
 
 def test_small_m_on_the_tile_kernel(fg, monkeypatch):
