@@ -187,11 +187,12 @@ FG8_API int fg_query_block_n(int M, int N, int K);
  *   layout 0 = normal (rows = M, G = 1), 1 = contiguous (rows = M_tot, G
  *   experts), 2 = masked (rows = M_max, G groups, expected_m as in the call).
  * Outputs (all required):
- *   *kernel_out  0 = the persistent tile kernel, 1 = the few-rows (decode) kernel
+ *   *kernel_out  0 = the tile kernel, 1 = the few-rows (decode) kernel
  *   *tile_n_out  BLOCK_N of the tile kernel, or the token-tile width of the
  *                decode kernel
  *   *pair_out    1 when tiles run on CTA pairs (256-row tiles)
- *   *splits_out  K splits per output tile (decode kernel; 1 otherwise)
+ *   *splits_out  K splits per output tile (decode kernel, or the tile kernel's
+ *                cluster split-K for few rows; 1 otherwise)
  *   *cluster_out CTAs per cluster (split-K reduction through distributed
  *                shared memory when equal to *splits_out > 1)
  * Returns FG_ERR_INVALID_ARG for a bad layout, non-positive sizes or a NULL
