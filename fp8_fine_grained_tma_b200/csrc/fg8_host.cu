@@ -629,7 +629,7 @@ fg_status get_streamk_workspace(int dev, cudaStream_t stream, size_t ws_bytes, s
 // token rows on the MMA's M side each promotion thread scales one row by two
 // scalars per K block (the swap-AB decode kernel needs a scale per column).
 // FG_TILE_SPLITK=0 / 1 forbids / forces it; by default it serves 64 < M <= 128
-// when the splits stay long (see below).
+// when the splits stay long enough (see splitk_plan).
 struct SplitKPlan {
     bool on = false;
     int bn = 0, ks = 0, ks_per = 0, tiles = 0;
@@ -647,14 +647,9 @@ cudaError_t max_split_clusters(int bn, int cluster, int* out) {
     }
 }
 
-SplitKPlan splitk_plan(int M, int N, int K, int sms) {
+// The largest resident split count for block width bn (0 when none >= 2).
+SplitKPlan splitk_for_width(int bn, int N, int KB, int sms) {
     SplitKPlan sp;
-    const char* env = std::getenv("FG_TILE_SPLITK");
-    const int mode = env ? std::atoi(env) : -1;
-    if (mode == 0 || M > BM) return sp;
-    if (mode < 0 && M <= 64) return sp;
-    const int KB = K / BK;
-    const int bn = N >= 256 ? 256 : (N + 15) / 16 * 16;
     const int tiles = (N + bn - 1) / bn;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -682,12 +677,6 @@ SplitKPlan splitk_plan(int M, int N, int K, int sms) {
             }
         }
         if (tiles <= mc) {
-            // Measured on B200 (M=128, back-to-back launches): against the
-            // swap-AB decode kernel this wins only when each split still has
-            // many K blocks (7168 x 16384: 34 vs 49 us, 32 K blocks per split)
-            // and loses with short splits (7 to 10 K blocks: 17 to 20 vs 13 to
-            // 17 us), where its set-up and the cluster reduction dominate.
-            if (mode < 0 && ks_per < 24) return sp;
             sp.on = true;
             sp.bn = bn;
             sp.ks = ks2;
@@ -697,6 +686,33 @@ SplitKPlan splitk_plan(int M, int N, int K, int sms) {
         }
     }
     return sp;
+}
+
+SplitKPlan splitk_plan(int M, int N, int K, int sms) {
+    SplitKPlan off;
+    const char* env = std::getenv("FG_TILE_SPLITK");
+    const int mode = env ? std::atoi(env) : -1;
+    if (mode == 0 || M > BM) return off;
+    if (mode < 0 && M <= 64) return off;
+    const int KB = K / BK;
+    const char* fbn_env = std::getenv("FG_FORCE_BLOCK_N");
+    const int fbn = fbn_env ? std::atoi(fbn_env) : 0;
+    if (fbn >= 16 && fbn <= 256 && fbn % 16 == 0) return splitk_for_width(fbn, N, KB, sms);
+    const int wide = N >= 256 ? 256 : (N + 15) / 16 * 16;
+    if (mode > 0) return splitk_for_width(wide, N, KB, sms);
+    // Measured on B200 (M=128, back-to-back launches) against the swap-AB
+    // decode kernel: 256-wide tiles win when every split keeps >= 24 K blocks
+    // (N=7168, K=16384: 34 vs 49 us); otherwise 128-wide tiles (twice the
+    // CTAs, four TMEM accumulators) win when a split keeps >= 8 K blocks
+    // (N=4096, K=7168: 15.5 vs 17 us; N=7168, K=2048: 12.9 vs 13.5 us); with
+    // shorter splits the set-up and the cluster reduction lose.
+    const SplitKPlan w = splitk_for_width(wide, N, KB, sms);
+    if (w.on && w.ks_per >= 24) return w;
+    if (N >= 256) {
+        const SplitKPlan h = splitk_for_width(128, N, KB, sms);
+        if (h.on && h.ks_per >= 8) return h;
+    }
+    return off;
 }
 
 fg_status run_gemm_splitk(const SplitKPlan& sp, const void* A, const float* sfa, const void* B, const float* sfb,

@@ -531,6 +531,24 @@ def test_tile_split_k_is_the_default_for_long_k_between_64_and_128_rows(fg, monk
     assert fg.query_plan("normal", 128, 7168, 16384)["kernel"] == "tile"
     assert fg.query_plan("normal", 64, 7168, 16384)["kernel"] == "decode"
     assert fg.query_plan("normal", 128, 2112, 7168)["kernel"] == "decode"
+    plan = fg.query_plan("normal", 128, 4096, 7168)
+    assert plan["kernel"] == "tile" and plan["tile_n"] == 128 and plan["splits"] >= 2
+
+
+def test_tile_split_k_128_wide_tiles_match_oracle(fg, monkeypatch):
+    """The default plan for M=128, N=4096, K=7168: 128-wide tiles (four TMEM
+    accumulators), K split over a cluster; every element against the oracle."""
+    monkeypatch.delenv("FG_TILE_SPLITK", raising=False)
+    monkeypatch.delenv("FG_FORCE_BLOCK_N", raising=False)
+    M, N, K = 128, 4096, 7168
+    assert fg.query_plan("normal", M, N, K)["tile_n"] == 128
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(4, 71))
+    A, sfa, B, sfb = to_gpu_normal(fg, x)
+    D = fg.fp8_gemm_nt(A, sfa, B, sfb)
+    torch.cuda.synchronize()
+    assert fg.get_last_device_status()[0] == 0
+    ref = oracle.gemm_nt(x.A.numpy(), x.sfa.numpy(), x.B.numpy(), x.sfb.numpy())
+    check(D.double().cpu().numpy(), ref)
 
 
 def test_small_m_on_the_tile_kernel(fg, monkeypatch):
