@@ -530,7 +530,7 @@ def test_tile_split_k_is_the_default_for_long_k_between_64_and_128_rows(fg, monk
     monkeypatch.delenv("FG_TILE_SPLITK", raising=False)
     assert fg.query_plan("normal", 128, 7168, 16384)["kernel"] == "tile"
     assert fg.query_plan("normal", 64, 7168, 16384)["kernel"] == "decode"
-    assert fg.query_plan("normal", 128, 2112, 7168)["kernel"] == "decode"
+    assert fg.query_plan("normal", 128, 7168, 2048)["kernel"] == "tile"
     plan = fg.query_plan("normal", 128, 4096, 7168)
     assert plan["kernel"] == "tile" and plan["tile_n"] == 128 and plan["splits"] >= 2
 
