@@ -14,10 +14,10 @@
 // all-zero block finite.
 //
 // B200 design: the op should be HBM-bound (5 bytes per FP32 element, 3 per
-// BF16), so the per-element work is kept to a few instructions: eight lanes
-// share a 128-element block (16 elements each, 16-byte coalesced loads, a
-// 3-step shuffle max, one 16-byte store of codes per lane) and a warp covers
-// four consecutive blocks per instruction.
+// BF16), so the per-element work is kept to a few instructions: a few lanes
+// share a 128-element block (16 or 32 elements each, 16-byte coalesced loads,
+// a short shuffle max, 16-byte stores of codes) and a warp covers four or
+// eight consecutive blocks per instruction.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -29,22 +29,33 @@ namespace fg8q {
 
 constexpr int QBLK = 128;
 constexpr int QTHREADS = 256;
-// Eight lanes quantise one 128-element block (16 elements each), so a warp
-// instruction serves four blocks: the per-block work (the amax reduction, the
-// scale, its reciprocal and the scale store) is shared four ways instead of
-// being paid once per 4 elements.  Latency is hidden by occupancy: 48 warps
-// per SM (six CTAs of 256 threads, at most 40 registers each), each with one
-// group of four blocks in flight, measured faster than fewer warps with two
-// groups each or with the next group prefetched.
-constexpr int QLANES = 8;
-constexpr int QEL = QBLK / QLANES;          // 16 elements per lane
-constexpr int QU = 1;
-constexpr int QMIN_BLOCKS = 6;
+// QL lanes quantise one 128-element block (QBLK / QL elements each), so a
+// warp instruction serves 32 / QL blocks: the per-block work (the amax
+// reduction, the scale, its reciprocal and the scale store) is shared by
+// that many blocks.  Latency is hidden by occupancy (MB CTAs of 256 threads
+// per SM), each warp with one group of blocks in flight.  Measured on B200 at
+// M=4096, K=7168: FP32 input is fastest with 8 lanes and six CTAs per SM
+// (0.87 of HBM; 4 lanes: 0.60), BF16 input with 4 lanes and four CTAs per SM
+// (0.61; 8 lanes: 0.55, 16 lanes: 0.43).  Two groups per warp in flight, or
+// the next group prefetched, were slower at both.
+template <typename T>
+struct QCfg;
+template <>
+struct QCfg<float> {
+    static constexpr int QL = 8;
+    static constexpr int MB = 6;
+};
+template <>
+struct QCfg<__nv_bfloat16> {
+    static constexpr int QL = 4;
+    static constexpr int MB = 4;
+};
 
-// 16 consecutive elements as FP32 (streaming loads: the input is read once).
-__device__ __forceinline__ void load16(const float* p, float (&v)[QEL]) {
+// QBLK / QL consecutive elements as FP32 (streaming loads: the input is read once).
+template <int N>
+__device__ __forceinline__ void load_elems(const float* p, float (&v)[N]) {
 #pragma unroll
-    for (int i = 0; i < QEL / 4; ++i) {
+    for (int i = 0; i < N / 4; ++i) {
         const float4 f = __ldcs(reinterpret_cast<const float4*>(p) + i);
         v[4 * i] = f.x;
         v[4 * i + 1] = f.y;
@@ -53,9 +64,10 @@ __device__ __forceinline__ void load16(const float* p, float (&v)[QEL]) {
     }
 }
 
-__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[QEL]) {
+template <int N>
+__device__ __forceinline__ void load_elems(const __nv_bfloat16* p, float (&v)[N]) {
 #pragma unroll
-    for (int i = 0; i < QEL / 8; ++i) {
+    for (int i = 0; i < N / 8; ++i) {
         const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p) + i);
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -102,56 +114,54 @@ __device__ __forceinline__ uint32_t to_e4m3x4(float a, float b, float c, float d
 }
 
 template <typename T>
-__global__ void __launch_bounds__(QTHREADS, QMIN_BLOCKS) quantize_kernel(const T* __restrict__ x, uint8_t* __restrict__ q,
-                                                            float* __restrict__ sfa, int M, int K, int m_pad) {
+__global__ void __launch_bounds__(QTHREADS, QCfg<T>::MB)
+    quantize_kernel(const T* __restrict__ x, uint8_t* __restrict__ q, float* __restrict__ sfa, int M, int K, int m_pad) {
+    constexpr int QL = QCfg<T>::QL;
+    constexpr int QEL = QBLK / QL;                  // elements per lane
+    constexpr int BPW = 32 / QL;                    // blocks per warp instruction
     const int KB = K / QBLK;
     const long long nblk = static_cast<long long>(M) * KB;
     const int lane = threadIdx.x % 32;
-    const int sub = lane / QLANES;                  // block of the warp's group of four
-    const int l8 = lane % QLANES;                   // 16-element slice of that block
+    const int sub = lane / QL;                      // block of the warp's group
+    const int ls = lane % QL;                       // slice of that block
     const long long warps = static_cast<long long>(gridDim.x) * (QTHREADS / 32);
     const long long w0 = static_cast<long long>(blockIdx.x) * (QTHREADS / 32) + threadIdx.x / 32;
-    const long long step = warps * 4;               // blocks per sweep of the whole grid
-    for (long long base = w0 * 4; base < nblk; base += step * QU) {
-        float v[QU][QEL];
+    const long long step = warps * BPW;             // blocks per sweep of the whole grid
+    for (long long base = w0 * BPW; base < nblk; base += step) {
+        const long long b = base + sub;
+        float v[QEL];
+        if (b < nblk) {
+            load_elems<QEL>(x + b * QBLK + ls * QEL, v);
+        } else {
 #pragma unroll
-        for (int u = 0; u < QU; ++u) {
-            const long long b = base + u * step + sub;
-            if (b < nblk) {
-                load16(x + b * QBLK + l8 * QEL, v[u]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < QEL; ++i) v[u][i] = 0.0f;
-            }
+            for (int i = 0; i < QEL; ++i) v[i] = 0.0f;
         }
+        float amax = 0.0f;
 #pragma unroll
-        for (int u = 0; u < QU; ++u) {
-            const long long b = base + u * step + sub;
-            float amax = 0.0f;
+        for (int i = 0; i < QEL; ++i) amax = fmaxf(amax, fabsf(v[i]));
 #pragma unroll
-            for (int i = 0; i < QEL; ++i) amax = fmaxf(amax, fabsf(v[u][i]));
+        for (int o = QL / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (b >= nblk) continue;
+        const float scale = fmaxf(amax, 1e-4f) / 448.0f;
+        const float rcp = __frcp_rn(scale);
+        uint32_t c[QEL / 4];
 #pragma unroll
-            for (int o = QLANES / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            if (b >= nblk) continue;
-            const float scale = fmaxf(amax, 1e-4f) / 448.0f;
-            const float rcp = __frcp_rn(scale);
-            uint32_t c[QEL / 4];
+        for (int i = 0; i < QEL / 4; ++i) {
+            const float2 lo = div_rn2(make_float2(v[4 * i], v[4 * i + 1]), scale, rcp);
+            const float2 hi = div_rn2(make_float2(v[4 * i + 2], v[4 * i + 3]), scale, rcp);
+            c[i] = to_e4m3x4(lo.x, lo.y, hi.x, hi.y);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(q + b * QBLK + ls * QEL);
 #pragma unroll
-            for (int i = 0; i < QEL / 4; ++i) {
-                const float2 lo = div_rn2(make_float2(v[u][4 * i], v[u][4 * i + 1]), scale, rcp);
-                const float2 hi = div_rn2(make_float2(v[u][4 * i + 2], v[u][4 * i + 3]), scale, rcp);
-                c[i] = to_e4m3x4(lo.x, lo.y, hi.x, hi.y);
-            }
-            __stcs(reinterpret_cast<uint4*>(q + b * QBLK + l8 * QEL), make_uint4(c[0], c[1], c[2], c[3]));
-            if (l8 == 0) {
-                // Block b is row m, K block kb (32-bit division whenever the
-                // block count allows it).
-                long long m;
-                if (nblk <= 0x7fffffffLL) m = static_cast<long long>(static_cast<unsigned>(b) / static_cast<unsigned>(KB));
-                else m = b / KB;
-                const int kb = static_cast<int>(b - m * KB);
-                sfa[static_cast<long long>(kb) * m_pad + m] = scale;
-            }
+        for (int i = 0; i < QEL / 16; ++i) __stcs(dst + i, make_uint4(c[4 * i], c[4 * i + 1], c[4 * i + 2], c[4 * i + 3]));
+        if (ls == 0) {
+            // Block b is row m, K block kb (32-bit division whenever the block
+            // count allows it).
+            long long m;
+            if (nblk <= 0x7fffffffLL) m = static_cast<long long>(static_cast<unsigned>(b) / static_cast<unsigned>(KB));
+            else m = b / KB;
+            const int kb = static_cast<int>(b - m * KB);
+            sfa[static_cast<long long>(kb) * m_pad + m] = scale;
         }
     }
     // Padding rows of the MN-major scales are zero.
@@ -199,17 +209,21 @@ extern "C" fg_status fg_quantize_fp8_activations(const void* x, int x_is_bf16, v
     if (sms <= 0) return FG_ERR_NO_DEVICE;
     const int m_pad = (M + 3) / 4 * 4;
     const long long nblk = static_cast<long long>(M) * (K / QBLK);
-    const long long warps_needed = (nblk + 4 * QU - 1) / (4 * QU);
-    const long long blocks_needed = (warps_needed + QTHREADS / 32 - 1) / (QTHREADS / 32);
-    const int grid = static_cast<int>(blocks_needed < static_cast<long long>(QMIN_BLOCKS) * sms ? (blocks_needed > 0 ? blocks_needed : 1)
-                                                                          : static_cast<long long>(QMIN_BLOCKS) * sms);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // One group of blocks per warp, capped at the resident grid.
+    auto grid_for = [&](int blocks_per_warp, int min_blocks) {
+        const long long warps_needed = (nblk + blocks_per_warp - 1) / blocks_per_warp;
+        const long long ctas = (warps_needed + QTHREADS / 32 - 1) / (QTHREADS / 32);
+        const long long cap = static_cast<long long>(min_blocks) * sms;
+        return static_cast<int>(ctas < cap ? (ctas > 0 ? ctas : 1) : cap);
+    };
     if (x_is_bf16)
-        quantize_kernel<__nv_bfloat16><<<grid, QTHREADS, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                                                 static_cast<uint8_t*>(q), sfa, M, K, m_pad);
+        quantize_kernel<__nv_bfloat16>
+            <<<grid_for(32 / QCfg<__nv_bfloat16>::QL, QCfg<__nv_bfloat16>::MB), QTHREADS, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(q), sfa, M, K, m_pad);
     else
-        quantize_kernel<float><<<grid, QTHREADS, 0, s>>>(static_cast<const float*>(x), static_cast<uint8_t*>(q), sfa,
-                                                         M, K, m_pad);
+        quantize_kernel<float><<<grid_for(32 / QCfg<float>::QL, QCfg<float>::MB), QTHREADS, 0, s>>>(
+            static_cast<const float*>(x), static_cast<uint8_t*>(q), sfa, M, K, m_pad);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? FG_OK : FG_ERR_CUDA;
 }
