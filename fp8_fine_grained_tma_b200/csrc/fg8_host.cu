@@ -892,7 +892,9 @@ fg_status fg_fp8_gemm_nt(const void* A, const float* sfa, const void* B, const f
         DeviceInfo* dev = nullptr;
         if (current_device(&dev) == FG_OK) {
             const SplitKPlan sp = splitk_plan(M, N, K, effective_sms(*dev));
-            if (sp.on) return run_gemm_splitk(sp, A, sfa, B, sfb, D, M, N, K, reinterpret_cast<cudaStream_t>(stream));
+            // A launch that is refused (nothing ran) falls back to the decode kernel.
+            if (sp.on && run_gemm_splitk(sp, A, sfa, B, sfb, D, M, N, K, reinterpret_cast<cudaStream_t>(stream)) == FG_OK)
+                return FG_OK;
         }
         return run_decode(A, sfa, B, sfb, D, M, N, K, reinterpret_cast<cudaStream_t>(stream));
     }
