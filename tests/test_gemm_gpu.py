@@ -535,14 +535,16 @@ def test_tile_split_k_is_the_default_for_long_k_between_64_and_128_rows(fg, monk
     assert plan["kernel"] == "tile" and plan["tile_n"] == 128 and plan["splits"] >= 2
 
 
-def test_tile_split_k_128_wide_tiles_match_oracle(fg, monkeypatch):
-    """The default plan for M=128, N=4096, K=7168: 128-wide tiles (four TMEM
-    accumulators), K split over a cluster; every element against the oracle."""
+@pytest.mark.parametrize("M,N,K", [(128, 4096, 7168), (100, 4112, 7168), (77, 7184, 2048)])
+def test_tile_split_k_128_wide_tiles_match_oracle(fg, M, N, K, monkeypatch):
+    """The default plan for few rows and moderate K: 128-wide tiles (four TMEM
+    accumulators), K split over a cluster, ragged M and a ragged last column
+    block; every element against the oracle."""
     monkeypatch.delenv("FG_TILE_SPLITK", raising=False)
     monkeypatch.delenv("FG_FORCE_BLOCK_N", raising=False)
-    M, N, K = 128, 4096, 7168
-    assert fg.query_plan("normal", M, N, K)["tile_n"] == 128
-    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(4, 71))
+    plan = fg.query_plan("normal", M, N, K)
+    assert plan["kernel"] == "tile" and plan["tile_n"] == 128 and plan["splits"] >= 2, plan
+    x = synth.normal_inputs(M, N, K, seed=synth.seed_for(4, 71) + M)
     A, sfa, B, sfb = to_gpu_normal(fg, x)
     D = fg.fp8_gemm_nt(A, sfa, B, sfb)
     torch.cuda.synchronize()
